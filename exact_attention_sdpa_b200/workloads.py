@@ -1,0 +1,115 @@
+"""Seeded synthetic inputs for the attention forward.
+
+This module only draws random numbers and fixes shapes; it holds none of the
+attention arithmetic, so both the CUDA path and the fp64 oracle can consume
+exactly the same input bits from it.
+
+Recipe (identical for every workload): a CPU ``torch.Generator`` seeded with
+the workload's seed draws fp32 standard-normal tensors in the fixed order
+q, k, v, bias, gate; each is multiplied by the workload's amplitude (a power
+of two, so the product is exact) and rounded to nearest-even into the
+workload's dtype.  Shapes follow the problem statement of the pages: Q, K, V
+and O are [B, H, N, d] with d contiguous (inskillml Module 9, the
+``scaled_dot_product_attention`` example), the Evoformer-style pair bias is
+[H, N, N] shared across the R rows that play the role of B, and the gate has
+O's shape (gist.science FLASHLIGHT summary, the gated row/column Evoformer
+variant).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional
+
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "algorithmic_bytes"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    dtype: str          # "fp16" | "bf16"
+    causal: bool
+    seed: int
+    amp: float = 1.0    # inputs are amp * N(0,1); a power of two keeps it exact
+    bias: bool = False  # additive pair bias [H, N, N], shared over B
+    gate: bool = False  # O <- sigmoid(G) * O, G has O's shape
+    description: str = ""
+
+    @property
+    def scale(self) -> float:
+        # 1/sqrt(d_k), aiinarabic.com "flash-attention", Equation (1)
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return {"fp16": torch.float16, "bf16": torch.bfloat16}[self.dtype]
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("tiny", B=1, H=2, N=256, d=64, dtype="bf16", causal=False, seed=0,
+                 description="tiny SDPA forward, B=1 H=2 N=256 d=64 bf16, non-causal"),
+        Workload("gpt2_small", B=4, H=12, N=1024, d=64, dtype="fp16", causal=True, seed=1,
+                 description="GPT-2-small-shaped attention, B=4 H=12 N=1024 d=64 fp16, causal"),
+        Workload("n8192_causal", B=4, H=12, N=8192, d=64, dtype="fp16", causal=True, seed=2,
+                 description="the inskillml Module 9 worked sizing, B=4 H=12 N=8192 d=64 fp16, causal"),
+        Workload("long_wide", B=1, H=32, N=32768, d=128, dtype="bf16", causal=True, seed=3, amp=0.5,
+                 description="long-context wide-head attention, B=1 H=32 N=32768 d=128 bf16 (x0.5), causal"),
+        Workload("evoformer_row", B=256, H=8, N=256, d=32, dtype="bf16", causal=False, seed=4,
+                 bias=True, gate=True,
+                 description="Evoformer-style gated row attention, R=256 H=8 N=256 d=32 bf16, "
+                             "pair bias [H,N,N], sigmoid gate"),
+    ]
+}
+
+
+def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional[torch.Tensor]]:
+    """Draw the workload's inputs on the CPU (see the module docstring for the recipe).
+
+    Returns a dict with keys q, k, v, bias, gate (bias/gate are None when the
+    workload has none).  Tensors are contiguous CPU tensors in the workload's
+    dtype; callers copy them to the device themselves.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    shape = (w.B, w.H, w.N, w.d)
+    dt = w.torch_dtype
+
+    def draw(*s):
+        x = torch.randn(*s, generator=g, dtype=torch.float32)
+        if w.amp != 1.0:
+            x.mul_(w.amp)
+        return x.to(dt)
+
+    q = draw(*shape)
+    k = draw(*shape)
+    v = draw(*shape)
+    bias = draw(w.H, w.N, w.N) if w.bias else None
+    gate = draw(*shape) if w.gate else None
+    return {"q": q, "k": k, "v": v, "bias": bias, "gate": gate}
+
+
+def attention_flops(w: Workload) -> float:
+    """The metric's FLOP count: 4*B*H*N^2*d, halved for causal."""
+    f = 4.0 * w.B * w.H * w.N * w.N * w.d
+    return f / 2.0 if w.causal else f
+
+
+def algorithmic_bytes(w: Workload) -> int:
+    """Bytes one forward must move at least once: Q, K, V (and G, bias) read, O and lse written."""
+    elem = 2
+    per_tensor = w.B * w.H * w.N * w.d * elem
+    n_tensors = 4 + (1 if w.gate else 0)          # q, k, v, o (+ gate)
+    bias = w.H * w.N * w.N * elem if w.bias else 0
+    lse = w.B * w.H * w.N * 4
+    return n_tensors * per_tensor + bias + lse

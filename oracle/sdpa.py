@@ -1,0 +1,154 @@
+"""fp64 CPU oracle for the exact scaled-dot-product attention forward.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may
+import or run this module.  It shares no code with the CUDA path and imports
+nothing from the ``exact_attention_sdpa_b200`` package.
+
+What it computes is the plain definition, because the fused method is exact
+(inskillml Module 9, "FlashAttention is not an approximation"; aiinarabic.com
+"flash-attention", the exactness remark beside the O(N^2) -> O(N) memory
+claim).  The definition is Equation (1) of aiinarabic.com "flash-attention",
+
+    Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V,
+
+evaluated row by row with the two-pass stable softmax that the gist.science
+FLASHLIGHT summary (Methodology, item 3, semantic fusion) names as the thing
+the online softmax replaces: pass 1 finds the row maximum, pass 2 sums the
+exponentials shifted by it.  Readings of points the pages leave open:
+
+* the explicit ``scale`` multiplies Q K^T, and the additive bias enters after
+  scaling: s = scale * q.k + bias;
+* causal: key j is visible to query i iff j <= i (square problems only);
+* lse_i = m_i + ln(l_i) in natural log, of the scaled, biased, masked scores;
+  the gate does not enter it;
+* the gate multiplies the normalised output elementwise by 1/(1+exp(-g));
+* a row whose every score is -inf has O = 0 and lse = -inf.
+
+Inputs of any float dtype are upcast exactly to float64 before any arithmetic.
+Parity: pinned (see tests/test_oracle.py for the pins).
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = ["sdpa_forward", "sdpa_rows", "to_f64"]
+
+
+def to_f64(x) -> Optional[np.ndarray]:
+    """Exact upcast of a torch tensor (fp16/bf16/fp32/fp64) or array to float64."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):                       # torch tensor, without importing torch here
+        x = x.detach().cpu()
+        if str(x.dtype) in ("torch.bfloat16", "torch.float16"):
+            x = x.float()                          # exact widening
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _bias_rows(bias: Optional[np.ndarray], b: int, h: int, rows: np.ndarray) -> Optional[np.ndarray]:
+    if bias is None:
+        return None
+    if bias.ndim == 3:                             # [H, Nq, Nk], shared over the batch (Evoformer pair bias)
+        return bias[h, rows, :]
+    return bias[b, h, rows, :]                     # [B, H, Nq, Nk]
+
+
+def _attend_rows(qr, k, v, bias_r, gate_r, rows, causal, scale) -> Tuple[np.ndarray, np.ndarray]:
+    """Two-pass stable softmax attention for a block of query rows of one (b, h).
+
+    qr: [r, d] queries; k, v: [Nk, d]; bias_r: [r, Nk] or None; rows: the
+    query indices of qr (for the causal mask).
+    """
+    # step 1: scores s_ij = scale * q_i . k_j (+ bias_ij), causal keys j > i masked to -inf
+    s = scale * (qr @ k.T)
+    if bias_r is not None:
+        s = s + bias_r
+    if causal:
+        keys = np.arange(k.shape[0])
+        s = np.where(keys[None, :] > rows[:, None], -np.inf, s)
+    # pass 1: row maximum
+    m = s.max(axis=1)
+    dead = ~np.isfinite(m) & (m < 0)               # every score of the row is -inf
+    m_safe = np.where(dead, 0.0, m)
+    # pass 2: shifted exponentials and their sum
+    w = np.exp(s - m_safe[:, None])
+    l = w.sum(axis=1)
+    # output = weighted mean of the value rows; logsumexp of the scores
+    with np.errstate(invalid="ignore", divide="ignore"):
+        o = (w @ v) / l[:, None]
+        lse = m + np.log(l)
+    o = np.where(dead[:, None], 0.0, o)
+    lse = np.where(dead, -np.inf, lse)
+    if gate_r is not None:
+        o = o * (1.0 / (1.0 + np.exp(-gate_r)))
+    return o, lse
+
+
+def _check(q, k, v, causal):
+    assert q.ndim == 4 and k.ndim == 4 and v.ndim == 4, "q, k, v must be [B, H, N, d]"
+    assert k.shape == v.shape and q.shape[:2] == k.shape[:2] and q.shape[3] == k.shape[3]
+    if causal:
+        assert q.shape[2] == k.shape[2], "causal masking is defined here for Nq == Nk"
+
+
+def sdpa_forward(q, k, v, bias=None, gate=None, causal: bool = False, scale: Optional[float] = None,
+                 block_rows: int = 1024) -> Tuple[np.ndarray, np.ndarray]:
+    """Full forward: returns (O [B,H,Nq,d], lse [B,H,Nq]) in float64.
+
+    q: [B,H,Nq,d]; k, v: [B,H,Nk,d]; bias: [H,Nq,Nk] or [B,H,Nq,Nk] or None;
+    gate: [B,H,Nq,d] or None; scale defaults to 1/sqrt(d).
+    Query rows are processed in blocks of ``block_rows`` only to bound memory.
+    """
+    q, k, v, bias, gate = (to_f64(t) for t in (q, k, v, bias, gate))
+    _check(q, k, v, causal)
+    B, H, Nq, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    O = np.zeros((B, H, Nq, d))
+    L = np.zeros((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, Nq, block_rows):
+                rows = np.arange(r0, min(Nq, r0 + block_rows))
+                o, lse = _attend_rows(q[b, h, rows], k[b, h], v[b, h], _bias_rows(bias, b, h, rows),
+                                      None if gate is None else gate[b, h, rows], rows, causal, scale)
+                O[b, h, rows] = o
+                L[b, h, rows] = lse
+    return O, L
+
+
+def sdpa_rows(q, k, v, picks: Sequence[Tuple[int, int, int]], bias=None, gate=None, causal: bool = False,
+              scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Selected output rows only: picks = [(b, h, i), ...]; returns (O [n,d], lse [n]) in float64.
+
+    Used to check full-size problems on a sample of rows; each row is computed
+    from the whole of its K, V exactly as in ``sdpa_forward``.
+    """
+    d = q.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out_o = np.zeros((len(picks), d))
+    out_l = np.zeros(len(picks))
+    by_bh = {}
+    for n, (b, h, i) in enumerate(picks):
+        by_bh.setdefault((b, h), []).append((n, i))
+    for (b, h), lst in by_bh.items():
+        idx = np.array([i for _, i in lst])
+        qr = to_f64(q[b, h][idx])
+        kb, vb = to_f64(k[b, h]), to_f64(v[b, h])
+        if causal:
+            assert q.shape[2] == k.shape[2]
+        br = None
+        if bias is not None:
+            bsel = bias[h] if bias.ndim == 3 else bias[b, h]
+            br = to_f64(bsel[idx])
+        gr = None if gate is None else to_f64(gate[b, h][idx])
+        o, lse = _attend_rows(qr, kb, vb, br, gr, idx, causal, scale)
+        for t, (n, _) in enumerate(lst):
+            out_o[n] = o[t]
+            out_l[n] = lse[t]
+    return out_o, out_l
