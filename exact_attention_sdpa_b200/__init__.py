@@ -1,0 +1,15 @@
+"""Exact fused scaled-dot-product attention forward for NVIDIA B200 (sm_100a).
+
+    from exact_attention_sdpa_b200 import attn_fwd
+    out, lse = attn_fwd(q, k, v, causal=True)
+
+The computation runs in ``libattn.so`` (built in-tree by
+``python -m exact_attention_sdpa_b200.build``); this package only marshals
+arguments.  Importing it does not load the library; the first call does, and
+raises if the library is missing.
+"""
+from ._native import (AttnError, attn_fwd, attn_fwd_raw, fwd, last_device_status, load_library,
+                      set_wait_limit, status_string, version)
+
+__all__ = ["attn_fwd", "attn_fwd_raw", "fwd", "AttnError", "last_device_status", "load_library",
+           "set_wait_limit", "status_string", "version"]

@@ -1,0 +1,294 @@
+// attn_api.cu -- the C ABI of libattn.so (declared in include/attn.h):
+// argument validation, TMA tensor-map encoding and kernel dispatch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace {
+
+using attn::FwdParams;
+
+__device__ unsigned int g_status_word;
+
+uint64_t g_wait_limit = 1ull << 32;
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+bool is_half_type(attn_dtype_t t) { return t == ATTN_F16 || t == ATTN_BF16; }
+
+int64_t span_bytes(const attn_tensor_t* t) {
+    // bytes from data to one past the last element (strides are non-negative)
+    int64_t last = 0;
+    for (int i = 0; i < t->ndim; ++i) last += (t->shape[i] - 1) * t->stride[i];
+    return (last + 1) * 2;
+}
+
+bool overlaps(const attn_tensor_t* a, const attn_tensor_t* b) {
+    if (a == nullptr || b == nullptr) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a->data), a1 = a0 + span_bytes(a);
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(b->data), b1 = b0 + span_bytes(b);
+    return a0 < b1 && b0 < a1;
+}
+
+// Common checks of a 16-bit tensor of rank `ndim`: positive shape, unit inner
+// stride, other strides positive multiples of 8 elements, 16-byte aligned data.
+attn_status_t check_tensor(const attn_tensor_t* t, int ndim) {
+    if (t == nullptr || t->data == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (t->ndim != ndim) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < ndim; ++i)
+        if (t->shape[i] <= 0) return ATTN_ERR_INVALID_ARG;
+    if (t->stride[ndim - 1] != 1) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < ndim - 1; ++i) {
+        if (t->stride[i] < 0 || (t->stride[i] % 8) != 0) return ATTN_ERR_INVALID_ARG;
+        if (t->shape[i] > 1 && t->stride[i] == 0) return ATTN_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(t->data) & 15u) != 0) return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+
+bool same_shape(const attn_tensor_t* a, const attn_tensor_t* b) {
+    if (a->ndim != b->ndim) return false;
+    for (int i = 0; i < a->ndim; ++i)
+        if (a->shape[i] != b->shape[i]) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps (driver entry point fetched through the runtime, so the library
+// does not link libcuda directly)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [B, H, N, d] view -> 4-D map with dims {d, N, H, B}, box {min(d,64), 128, 1, 1}
+bool encode_qkv_map(CUtensorMap* map, const attn_tensor_t* t) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (enc == nullptr) return false;
+    const int64_t d = t->shape[3];
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)t->shape[2], (cuuint64_t)t->shape[1],
+                                (cuuint64_t)t->shape[0]};
+    // a stride of a size-1 dimension is irrelevant; give TMA a legal one
+    auto stride_or = [&](int i, int64_t fallback) { return t->shape[i] > 1 ? t->stride[i] : fallback; };
+    const int64_t sN = stride_or(2, d);
+    const int64_t sH = stride_or(1, sN * t->shape[2]);
+    const int64_t sB = stride_or(0, sH * t->shape[1]);
+    const cuuint64_t strides[3] = {(cuuint64_t)(sN * 2), (cuuint64_t)(sH * 2), (cuuint64_t)(sB * 2)};
+    const cuuint32_t box[4] = {(cuuint32_t)(d >= 64 ? 64 : d), 128u, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUtensorMapDataType dt =
+        t->dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapSwizzle sw = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return enc(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// dispatch
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE>
+cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+                     cudaStream_t stream) {
+    auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE>;
+    constexpr int smem = attn::FwdSmem<D>::kDynBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<p.num_units, attn::kThreads, smem, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_d(bool causal, bool bias, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const FwdParams& p, cudaStream_t s) {
+#define ATTN_CASE(C, B_, G_) \
+    if (causal == C && bias == B_ && gate == G_) return launch_t<T, D, C, B_, G_>(mq, mk, mv, p, s);
+    ATTN_CASE(false, false, false)
+    ATTN_CASE(false, false, true)
+    ATTN_CASE(false, true, false)
+    ATTN_CASE(false, true, true)
+    ATTN_CASE(true, false, false)
+    ATTN_CASE(true, false, true)
+    ATTN_CASE(true, true, false)
+    ATTN_CASE(true, true, true)
+#undef ATTN_CASE
+    return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t launch_dtype(int d, bool causal, bool bias, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const FwdParams& p, cudaStream_t s) {
+    switch (d) {
+        case 32: return launch_d<T, 32>(causal, bias, gate, mq, mk, mv, p, s);
+        case 64: return launch_d<T, 64>(causal, bias, gate, mq, mk, mv, p, s);
+        case 128: return launch_d<T, 128>(causal, bias, gate, mq, mk, mv, p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+unsigned int* status_word_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    static unsigned int* ptrs[64] = {nullptr};
+    static std::mutex mu;
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<unsigned int*>(ptr);
+    }
+    return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                       attn_tensor_t* out, float* lse, cudaStream_t stream) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+    // dtype rules first: fp32 is a valid request this fused kernel does not serve
+    if (q->dtype == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+    if (!is_half_type(q->dtype)) return ATTN_ERR_INVALID_ARG;
+    if (k->dtype != q->dtype || v->dtype != q->dtype || out->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
+    if (bias != nullptr && bias->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
+    if (gate != nullptr && gate->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+
+    // empty problems: nothing to do
+    if (q->ndim == 4 && (q->shape[0] == 0 || q->shape[1] == 0 || q->shape[2] == 0)) {
+        if (k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return ATTN_ERR_INVALID_ARG;
+        if (!same_shape(q, k) || !same_shape(q, v) || !same_shape(q, out)) return ATTN_ERR_INVALID_ARG;
+        return ATTN_OK;
+    }
+    attn_status_t st;
+    if ((st = check_tensor(q, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(k, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(v, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(out, 4)) != ATTN_OK) return st;
+    if (!same_shape(q, k) || !same_shape(q, v) || !same_shape(q, out)) return ATTN_ERR_INVALID_ARG;
+    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], d = q->shape[3];
+    if (d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (N > (int64_t(1) << 30) || B * H > (int64_t(1) << 24)) return ATTN_ERR_UNSUPPORTED;
+    if (gate != nullptr) {
+        if ((st = check_tensor(gate, 4)) != ATTN_OK) return st;
+        if (!same_shape(q, gate)) return ATTN_ERR_INVALID_ARG;
+    }
+    if (bias != nullptr) {
+        if (bias->ndim == 3) {
+            if ((st = check_tensor(bias, 3)) != ATTN_OK) return st;
+            if (bias->shape[0] != H || bias->shape[1] != N || bias->shape[2] != N) return ATTN_ERR_INVALID_ARG;
+        } else if (bias->ndim == 4) {
+            if ((st = check_tensor(bias, 4)) != ATTN_OK) return st;
+            if (bias->shape[0] != B || bias->shape[1] != H || bias->shape[2] != N || bias->shape[3] != N)
+                return ATTN_ERR_INVALID_ARG;
+        } else {
+            return ATTN_ERR_INVALID_ARG;
+        }
+    }
+    if (overlaps(out, q) || overlaps(out, k) || overlaps(out, v) || overlaps(out, bias) || overlaps(out, gate))
+        return ATTN_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+
+    // ---- launch
+    CUtensorMap mq, mk, mv;
+    if (!encode_qkv_map(&mq, q) || !encode_qkv_map(&mk, k) || !encode_qkv_map(&mv, v)) return ATTN_ERR_CUDA;
+    unsigned int* status = status_word_ptr();
+    if (status == nullptr) return ATTN_ERR_CUDA;
+
+    FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = static_cast<int>(B);
+    p.H = static_cast<int>(H);
+    p.N = static_cast<int>(N);
+    p.num_q_tiles = static_cast<int>((N + attn::kBlockM - 1) / attn::kBlockM);
+    const int64_t units = static_cast<int64_t>(p.num_q_tiles) * B * H;
+    if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    p.num_units = static_cast<int>(units);
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    if (bias != nullptr) {
+        p.bias = bias->data;
+        if (bias->ndim == 3) {
+            p.bias_sb = 0;
+            p.bias_sh = bias->stride[0];
+            p.bias_si = bias->stride[1];
+        } else {
+            p.bias_sb = bias->stride[0];
+            p.bias_sh = bias->stride[1];
+            p.bias_si = bias->stride[2];
+        }
+    }
+    if (gate != nullptr) {
+        p.gate = gate->data;
+        p.gate_sb = gate->stride[0];
+        p.gate_sh = gate->stride[1];
+        p.gate_si = gate->stride[2];
+    }
+    p.out = out->data;
+    p.out_sb = out->stride[0];
+    p.out_sh = out->stride[1];
+    p.out_si = out->stride[2];
+    p.lse = lse;
+    p.wait_limit = g_wait_limit;
+    p.status = status;
+
+    cudaError_t e;
+    if (q->dtype == ATTN_BF16)
+        e = launch_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, mq, mk,
+                                        mv, p, stream);
+    else
+        e = launch_dtype<__half>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, mq, mk, mv,
+                                 p, stream);
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+const char* attn_status_string(attn_status_t status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument (null, shape/stride mismatch, misalignment, aliasing or non-finite scale)";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported (fp32, mixed dtypes, or head dim not in {32, 64, 128})";
+        case ATTN_ERR_CUDA: return "CUDA error (launch, tensor-map encoding or device query failed)";
+        case ATTN_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+attn_status_t attn_last_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    unsigned int* ptr = status_word_ptr();
+    if (ptr == nullptr) return ATTN_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+    const unsigned int zero = 0;
+    if (cudaMemcpy(ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+    return (v & attn::kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+void attn_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles < 1024 ? 1024 : cycles; }
+
+const char* attn_version(void) { return "0.1.0"; }
+
+}  // extern "C"

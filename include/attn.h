@@ -1,0 +1,127 @@
+/*
+ * attn.h -- C ABI of libattn.so: the fused, exact scaled-dot-product attention
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * Operation (aiinarabic.com "flash-attention", Equation (1), with the optional
+ * additive bias and sigmoid gate of the gated Evoformer variant named in the
+ * gist.science FLASHLIGHT summary):
+ *
+ *     S   = scale * Q K^T (+ bias),   S_ij = -inf for j > i when causal
+ *     O   = softmax_rows(S) V   (then O <- O * sigmoid(G) when a gate is given)
+ *     lse = per-row natural-log logsumexp of S, i.e. m + ln(l) for the row
+ *           maximum m and the sum l of exp(S - m); the gate does not enter it.
+ *
+ * It is computed block by block with an online softmax (running max and
+ * running sum, the sum rescaled by e^(m_old - m_new) when the max grows; the
+ * gist.science FLASHLIGHT summary, Methodology item 3), so the N x N score
+ * matrix never reaches global memory (aiinarabic.com "flash-attention", the
+ * kernel-fusion and tiling sections).  lse is the per-row normaliser that a
+ * backward pass needs to recompute the softmax (the same page, recomputation).
+ *
+ * Threading and ownership: the caller owns every buffer.  The library keeps no
+ * per-call allocations; it caches nothing but an internal device status word.
+ * All calls are asynchronous on `stream` and never synchronise it (except
+ * attn_last_device_status, which says so).  Outputs are valid once `stream`
+ * reaches the call.
+ */
+#ifndef ATTN_B200_ATTN_H_
+#define ATTN_B200_ATTN_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,   /* null pointer, shape/stride mismatch, misalignment, non-finite scale */
+    ATTN_ERR_UNSUPPORTED = 2,   /* a valid request this kernel does not implement (fp32, head dim, ...) */
+    ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call or the launch failed */
+    ATTN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (status word, see below) */
+} attn_status_t;
+
+typedef enum {
+    ATTN_F16 = 0,
+    ATTN_BF16 = 1,
+    ATTN_F32 = 2                /* accepted by the type only so that it can be rejected (UNSUPPORTED) */
+} attn_dtype_t;
+
+/*
+ * A strided view of a device tensor.  shape and stride are in ELEMENTS, outer
+ * to inner; only the first `ndim` entries are read.  Q, K, V, O and the gate
+ * are 4-D [B, H, N, d]; the innermost stride must be 1 and every other stride
+ * times the element size must be a multiple of 16 bytes, and `data` must be
+ * 16-byte aligned (tensor-memory-accelerator copies need both).
+ */
+typedef struct {
+    void* data;
+    attn_dtype_t dtype;
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];
+} attn_tensor_t;
+
+/*
+ * attn_fwd -- O = softmax(scale * Q K^T [+ bias]) V [* sigmoid(G)] and lse.
+ *
+ *   q       [B, H, N, d]  fp16 or bf16, device memory.
+ *   k, v    [B, H, N, d]  same dtype, B, H, N and d as q.
+ *   bias    nullable.  Additive score bias of q's dtype, either [H, N, N]
+ *           (shared over B, the Evoformer pair bias) or [B, H, N, N]; the
+ *           innermost stride must be 1 and rows 16-byte aligned.
+ *   gate    nullable.  [B, H, N, d] of q's dtype; O is multiplied elementwise
+ *           by 1/(1+exp(-gate)) after normalisation.
+ *   causal  nonzero: key j is visible to query i iff j <= i.
+ *   scale   multiplies Q K^T; must be finite (0 is legal).  Callers normally
+ *           pass 1/sqrt(d).
+ *   out     [B, H, N, d] of q's dtype, written (fp32 accumulator rounded to
+ *           nearest even).  Must not alias q, k, v, bias or gate.
+ *   lse     nullable.  B*H*N contiguous fp32, row (b, h, i) at (b*H + h)*N + i,
+ *           natural log.  A row with every score -inf gets O = 0, lse = -inf.
+ *   stream  CUDA stream of the launch (0 = legacy default stream).
+ *
+ * Supported: d in {32, 64, 128}; N >= 1 (any N, ragged tails are masked);
+ * B*H >= 1.  N == 0 or B*H == 0 returns ATTN_OK without launching.
+ * Errors are detected on the host before any launch and return a status with
+ * no side effect: ATTN_ERR_INVALID_ARG for nulls, rank/shape/stride mismatch,
+ * misalignment, aliasing of out with an input, or a non-finite scale;
+ * ATTN_ERR_UNSUPPORTED for fp32, mixed dtypes, or d outside {32, 64, 128};
+ * ATTN_ERR_CUDA if the launch fails.
+ */
+attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* bias, const attn_tensor_t* gate,
+                       int causal, float scale,
+                       attn_tensor_t* out, float* lse,
+                       cudaStream_t stream);
+
+/* A static, NUL-terminated description of a status code (never NULL). */
+const char* attn_status_string(attn_status_t status);
+
+/*
+ * attn_last_device_status -- synchronises `stream`, then reads and clears the
+ * device status word of the current device.  Kernels bound every wait on an
+ * mbarrier; a wait that gives up records ATTN_ERR_TIMEOUT there (and the
+ * kernel returns without hanging).  Returns ATTN_OK, ATTN_ERR_TIMEOUT, or
+ * ATTN_ERR_CUDA if synchronising or reading failed.
+ */
+attn_status_t attn_last_device_status(cudaStream_t stream);
+
+/*
+ * attn_set_wait_limit -- sets the clock-cycle budget of every bounded device
+ * wait for later launches on the current device (default 2^32 cycles, about
+ * two seconds at 1.9 GHz).  Values below 1024 are raised to 1024.  Tests use a
+ * small limit to exercise the timeout path without a fault.  Not thread-safe
+ * with concurrent attn_fwd calls.
+ */
+void attn_set_wait_limit(uint64_t cycles);
+
+/* The library version as "major.minor.patch" (static string). */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_ATTN_H_ */

@@ -1,0 +1,186 @@
+"""Host-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments with the documented status codes
+before touching the GPU (so these run without one)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from exact_attention_sdpa_b200 import _native as nat
+from exact_attention_sdpa_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return nat.load_library()
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_binding_surface():
+    assert set(_declared_functions()) == set(nat.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", nat.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (attn_\w+)", out))
+    for name in _declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        s = nat.status_string(code)
+        assert isinstance(s, str) and len(s) > 0
+    assert nat.status_string(123) == "unknown status"
+    assert nat.version().count(".") == 2
+
+
+def _qkv(B=1, H=2, N=64, d=64, dtype=torch.float16):
+    # CPU tensors: only their addresses/shapes are read by the host-side checks
+    mk = lambda: torch.zeros(B, H, N, d, dtype=dtype)
+    return mk(), mk(), mk(), mk()
+
+
+def call(q, k, v, out, bias=None, gate=None, causal=False, scale=0.125, lse=None):
+    return nat.attn_fwd_raw(q, k, v, bias, gate, causal, scale, out, lse, 0)
+
+
+def test_null_arguments(lib):
+    q, k, v, o = _qkv()
+    P = ctypes.POINTER(nat.AttnTensor)
+    vq, vk, vv, vo = (nat.make_view(t) for t in (q, k, v, o))
+    r = lib.attn_fwd(None, ctypes.byref(vk), ctypes.byref(vv), None, None, 0, 0.1, ctypes.byref(vo), None, None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+    r = lib.attn_fwd(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), None, None, 0, 0.1, None, None, None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+    vq.data = None
+    r = lib.attn_fwd(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), None, None, 0, 0.1, ctypes.byref(vo),
+                     None, None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_fp32_is_unsupported(lib):
+    q, k, v, o = _qkv(dtype=torch.float32)
+    assert call(q, k, v, o) == nat.ATTN_ERR_UNSUPPORTED
+
+
+def test_mixed_dtypes_unsupported(lib):
+    q, k, v, o = _qkv()
+    assert call(q, k.to(torch.bfloat16), v, o) == nat.ATTN_ERR_UNSUPPORTED
+    assert call(q, k, v, o.to(torch.bfloat16)) == nat.ATTN_ERR_UNSUPPORTED
+
+
+def test_unknown_dtype_invalid(lib):
+    q, k, v, o = _qkv()
+    assert call(q.to(torch.int16), k, v, o) == nat.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [16, 48, 96, 256])
+def test_head_dim_unsupported(lib, d):
+    q, k, v, o = _qkv(d=d)
+    assert call(q, k, v, o) == nat.ATTN_ERR_UNSUPPORTED
+
+
+def test_shape_mismatch(lib):
+    q, k, v, o = _qkv()
+    k2 = torch.zeros(1, 2, 65, 64, dtype=torch.float16)
+    assert call(q, k2, v, o) == nat.ATTN_ERR_INVALID_ARG
+    o2 = torch.zeros(1, 3, 64, 64, dtype=torch.float16)
+    assert call(q, k, v, o2) == nat.ATTN_ERR_INVALID_ARG
+    assert call(q[0], k[0], v[0], o[0]) == nat.ATTN_ERR_INVALID_ARG          # rank 3
+
+
+def test_non_unit_inner_stride(lib):
+    q, k, v, o = _qkv()
+    qt = torch.zeros(1, 2, 64, 64, dtype=torch.float16).transpose(2, 3)
+    assert call(qt, k, v, o) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_misaligned_row_stride(lib):
+    # rows 68 elements apart (136 bytes): not a multiple of 16 bytes
+    base = torch.zeros(1, 2, 64, 68, dtype=torch.float16)
+    q = base[..., :64]
+    _, k, v, o = _qkv()
+    assert call(q, k, v, o) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_misaligned_base(lib):
+    flat = torch.zeros(1 * 2 * 64 * 64 + 8, dtype=torch.float16)
+    q = flat[1:1 + 2 * 64 * 64].view(1, 2, 64, 64)                            # 2-byte offset
+    _, k, v, o = _qkv()
+    assert call(q, k, v, o) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_non_finite_scale(lib):
+    q, k, v, o = _qkv()
+    assert call(q, k, v, o, scale=float("nan")) == nat.ATTN_ERR_INVALID_ARG
+    assert call(q, k, v, o, scale=float("inf")) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_out_aliasing_input(lib):
+    q, k, v, _ = _qkv()
+    assert call(q, k, v, q) == nat.ATTN_ERR_INVALID_ARG
+    assert call(q, k, v, v) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_bias_and_gate_shapes(lib):
+    q, k, v, o = _qkv()
+    bad_bias = torch.zeros(2, 64, 32, dtype=torch.float16)
+    assert call(q, k, v, o, bias=bad_bias) == nat.ATTN_ERR_INVALID_ARG
+    bad_bias4 = torch.zeros(2, 2, 64, 64, dtype=torch.float16)               # B mismatch
+    assert call(q, k, v, o, bias=bad_bias4) == nat.ATTN_ERR_INVALID_ARG
+    assert call(q, k, v, o, bias=torch.zeros(64, 64, dtype=torch.float16)) == nat.ATTN_ERR_INVALID_ARG
+    assert call(q, k, v, o, bias=torch.zeros(2, 64, 64, dtype=torch.bfloat16)) == nat.ATTN_ERR_UNSUPPORTED
+    bad_gate = torch.zeros(1, 2, 64, 32, dtype=torch.float16)
+    assert call(q, k, v, o, gate=bad_gate) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_misaligned_lse(lib):
+    q, k, v, o = _qkv()
+    lse = torch.zeros(1 + 2 * 64, dtype=torch.uint8)[1:]
+    r = nat.attn_fwd_raw(q, k, v, None, None, False, 0.1, o, None, 0)
+    vq, vk, vv, vo = (nat.make_view(t) for t in (q, k, v, o))
+    r = nat.load_library().attn_fwd(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), None, None, 0, 0.1,
+                                    ctypes.byref(vo), lse.data_ptr(), None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_empty_problem_is_ok_without_launch(lib):
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
+    assert call(q, q.clone(), q.clone(), q.clone()) == nat.ATTN_OK
+    q = torch.zeros(0, 2, 16, 64, dtype=torch.float16)
+    assert call(q, q.clone(), q.clone(), q.clone()) == nat.ATTN_OK
+    k = torch.zeros(1, 2, 3, 64, dtype=torch.float16)
+    assert call(torch.zeros(1, 2, 0, 64, dtype=torch.float16), k, k, k) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no fallback"):
+        nat.load_library(str(tmp_path / "libattn.so"))
+
+
+def test_product_path_does_not_reach_the_oracle():
+    # no import of, or path into, the oracle package anywhere in the product
+    pat = re.compile(r"^\s*(from\s+oracle\b|import\s+oracle\b)|oracle/|importlib.*oracle", re.M)
+    pkg = os.path.join(ROOT, "exact_attention_sdpa_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not pat.search(text), fn

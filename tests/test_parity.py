@@ -1,0 +1,128 @@
+"""GPU parity: the fused sm_100a kernel against the fp64 oracle on the same
+seeded inputs (element by element), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_sdpa_b200 import attn_fwd
+from exact_attention_sdpa_b200.workloads import WORKLOADS, Workload, make_inputs
+from oracle import sdpa_forward, sdpa_rows
+from helpers import assert_close_to_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, w: Workload, scale=None):
+    dev = torch.device("cuda")
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    bias = None if inp["bias"] is None else inp["bias"].to(dev)
+    gate = None if inp["gate"] is None else inp["gate"].to(dev)
+    o, lse = attn_fwd(q, k, v, bias=bias, gate=gate, causal=w.causal, scale=w.scale if scale is None else scale)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def _full_check(w: Workload, seed=None):
+    inp = make_inputs(w, seed)
+    o, lse = _run(inp, w)
+    o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], bias=inp["bias"], gate=inp["gate"],
+                                causal=w.causal, scale=w.scale)
+    return assert_close_to_oracle(o, lse, o_ref, l_ref, w.torch_dtype, w.name)
+
+
+@pytest.mark.parametrize("name", ["tiny", "gpt2_small", "evoformer_row"])
+def test_workload_full(name):
+    _full_check(WORKLOADS[name])
+
+
+def _sampled_rows(w: Workload, n_bh=4, seed=0):
+    """Rows every query tile boundary cares about, plus random ones, for a few (b, h)."""
+    rng = np.random.default_rng(seed)
+    picks = []
+    bhs = [(0, 0), (w.B - 1, w.H - 1)] + [(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(n_bh - 2)]
+    special = [0, 1, 127, 128, 129, w.N // 2, w.N - 129, w.N - 128, w.N - 2, w.N - 1]
+    for b, h in bhs:
+        rows = set(i for i in special if 0 <= i < w.N)
+        rows.update(int(x) for x in rng.integers(0, w.N, size=24))
+        picks += [(b, h, i) for i in sorted(rows)]
+    return picks
+
+
+@pytest.mark.parametrize("name", ["n8192_causal", "long_wide"])
+def test_workload_full_size_sampled(name):
+    """Full-size problems in the launch configuration the benchmark times;
+    the oracle computes a sample of output rows one by one."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    o, lse = _run(inp, w)
+    picks = _sampled_rows(w)
+    o_ref, l_ref = sdpa_rows(inp["q"], inp["k"], inp["v"], picks, bias=inp["bias"], gate=inp["gate"],
+                             causal=w.causal, scale=w.scale)
+    idx = tuple(np.array(x) for x in zip(*picks))
+    o_s = o.cpu()[idx]
+    l_s = lse.cpu()[idx]
+    assert_close_to_oracle(o_s, l_s, o_ref, l_ref, w.torch_dtype, name)
+    # every output row (not only the sampled ones) is finite
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+SWEEP = []
+for d in (32, 64, 128):
+    for N in (1, 17, 128, 129, 255, 1000):
+        for causal in (False, True):
+            SWEEP.append((d, N, causal))
+
+
+@pytest.mark.parametrize("d,N,causal", SWEEP)
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_sweep_ragged(d, N, causal, dtype):
+    w = Workload("sweep", B=1, H=3, N=N, d=d, dtype=dtype, causal=causal, seed=100 + d + N)
+    _full_check(w)
+
+
+@pytest.mark.parametrize("bias,gate", [(True, False), (False, True), (True, True)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d,N", [(32, 200), (64, 256), (128, 129)])
+def test_bias_gate_variants(bias, gate, causal, d, N):
+    w = Workload("bg", B=3, H=2, N=N, d=d, dtype="bf16", causal=causal, seed=7 + N, bias=bias, gate=gate)
+    _full_check(w)
+
+
+def test_per_batch_bias_4d():
+    w = Workload("b4", B=2, H=3, N=300, d=64, dtype="fp16", causal=False, seed=11)
+    inp = make_inputs(w)
+    bias = torch.randn(2, 3, 300, 304, generator=torch.Generator().manual_seed(5)).to(torch.float16)[..., :300]
+    dev = torch.device("cuda")
+    o, lse = attn_fwd(inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev), bias=bias.to(dev), causal=False,
+                      scale=w.scale)
+    o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], bias=bias, scale=w.scale)
+    assert_close_to_oracle(o, lse, o_ref, l_ref, torch.float16, "bias4d")
+
+
+def test_strided_views():
+    """Q/K/V as transposed views of [B, N, H, d] buffers; O written into a strided view."""
+    B, H, N, d = 2, 4, 333, 64
+    g = torch.Generator().manual_seed(3)
+    mk = lambda: torch.randn(B, N, H, d, generator=g).to(torch.bfloat16)
+    qb, kb, vb = mk(), mk(), mk()
+    dev = torch.device("cuda")
+    q, k, v = (x.to(dev).transpose(1, 2) for x in (qb, kb, vb))
+    out_buf = torch.zeros(B, N, H, d, device=dev, dtype=torch.bfloat16)
+    out = out_buf.transpose(1, 2)
+    _, lse = attn_fwd(q, k, v, causal=True, out=out)
+    torch.cuda.synchronize()
+    o_ref, l_ref = sdpa_forward(qb.transpose(1, 2), kb.transpose(1, 2), vb.transpose(1, 2), causal=True)
+    assert_close_to_oracle(out_buf.transpose(1, 2), lse, o_ref, l_ref, torch.bfloat16, "strided")
+
+
+def test_deterministic():
+    w = WORKLOADS["gpt2_small"]
+    inp = make_inputs(w)
+    o1, l1 = _run(inp, w)
+    o2, l2 = _run(inp, w)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_batch_heads_many():
+    w = Workload("bh", B=5, H=7, N=160, d=64, dtype="fp16", causal=True, seed=21)
+    _full_check(w)
