@@ -33,3 +33,15 @@ def assert_close_to_oracle(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
         lerr = np.abs(l[fin] - lse_ref[fin])
         assert np.all(lerr <= tol), f"{what}: lse err {float(lerr.max()):.3e} exceeds 1e-3 relative"
     return worst
+
+
+def padded(t: torch.Tensor, device=None) -> torch.Tensor:
+    """The same values, on ``device``, stored with the last dimension padded to a
+    multiple of 8 elements (16 bytes), as the C ABI requires of bias rows.
+    (The padding buffer is created on the target device because copying a
+    non-dense view across devices would make it contiguous again.)"""
+    n = t.shape[-1]
+    device = t.device if device is None else torch.device(device)
+    buf = torch.zeros(*t.shape[:-1], (n + 7) // 8 * 8, dtype=t.dtype, device=device)
+    buf[..., :n] = t.to(device)
+    return buf[..., :n]

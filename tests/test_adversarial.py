@@ -9,7 +9,7 @@ import torch
 
 from exact_attention_sdpa_b200 import attn_fwd
 from oracle import sdpa_forward
-from helpers import assert_close_to_oracle
+from helpers import assert_close_to_oracle, padded
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda") if torch.cuda.is_available() else None
@@ -23,7 +23,7 @@ def _gen(shape, seed, dtype, scale=1.0):
 def _check(q, k, v, bias=None, gate=None, causal=False, scale=None, what=""):
     d = q.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    o, lse = attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), None if bias is None else bias.to(DEV),
+    o, lse = attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), None if bias is None else padded(bias, DEV),
                       None if gate is None else gate.to(DEV), causal=causal, scale=scale)
     torch.cuda.synchronize()
     o_ref, l_ref = sdpa_forward(q, k, v, bias=bias, gate=gate, causal=causal, scale=scale)

@@ -7,7 +7,7 @@ import torch
 from exact_attention_sdpa_b200 import attn_fwd
 from exact_attention_sdpa_b200.workloads import WORKLOADS, Workload, make_inputs
 from oracle import sdpa_forward, sdpa_rows
-from helpers import assert_close_to_oracle
+from helpers import assert_close_to_oracle, padded
 
 pytestmark = pytest.mark.gpu
 
@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 def _run(inp, w: Workload, scale=None):
     dev = torch.device("cuda")
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
-    bias = None if inp["bias"] is None else inp["bias"].to(dev)
+    bias = None if inp["bias"] is None else padded(inp["bias"], dev)
     gate = None if inp["gate"] is None else inp["gate"].to(dev)
     o, lse = attn_fwd(q, k, v, bias=bias, gate=gate, causal=w.causal, scale=w.scale if scale is None else scale)
     torch.cuda.synchronize()
@@ -93,7 +93,7 @@ def test_per_batch_bias_4d():
     inp = make_inputs(w)
     bias = torch.randn(2, 3, 300, 304, generator=torch.Generator().manual_seed(5)).to(torch.float16)[..., :300]
     dev = torch.device("cuda")
-    o, lse = attn_fwd(inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev), bias=bias.to(dev), causal=False,
+    o, lse = attn_fwd(inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev), bias=padded(bias, dev), causal=False,
                       scale=w.scale)
     o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], bias=bias, scale=w.scale)
     assert_close_to_oracle(o, lse, o_ref, l_ref, torch.float16, "bias4d")
