@@ -164,6 +164,36 @@ def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
     return flops / secs / 1e12, sample, cores
 
 
+def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
+    """The same metric through fwd(): every step copies the step's inputs from
+    pinned host memory to the device, runs the kernel, and reads O and lse back."""
+    from exact_attention_sdpa_b200 import fwd
+    host = {k: (None if t is None else t.pin_memory()) for k, t in inp_cpu.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = out.numel() * out.element_size() + lse.numel() * 4
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e_step():
+        fwd(host["q"], host["k"], host["v"], bias=host["bias"], gate=host["gate"], causal=w.causal, scale=w.scale,
+            out=out_h, lse=lse_h)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = dist_max(e0.elapsed_time(e1) / steps, world)
+    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -173,6 +203,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=8)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-staged end-to-end leg (profiling runs)")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     flops = attention_flops(w)
@@ -197,7 +228,7 @@ def main():
         return
 
     world, rank, local = dist_setup(args.gpus)
-    from exact_attention_sdpa_b200 import attn_fwd, fwd, load_library
+    from exact_attention_sdpa_b200 import attn_fwd, load_library
     load_library()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -236,29 +267,7 @@ def main():
     value = world * flops / (ms_per_step * 1e-3) / 1e12
 
     # ---- end to end through the public API: pinned host inputs in, host outputs back, every step
-    host = {k: (None if t is None else t.pin_memory()) for k, t in inp_cpu.items()}
-    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
-    d2h = out.numel() * out.element_size() + lse.numel() * 4
-    e2e_steps = max(3, min(args.steps, 20))
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-
-    def e2e_step():
-        fwd(host["q"], host["k"], host["v"], bias=host["bias"], gate=host["gate"], causal=w.causal, scale=w.scale,
-            out=out_h, lse=lse_h)
-
-    for _ in range(2):
-        e2e_step()
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = dist_max(e0.elapsed_time(e1) / e2e_steps, world)
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    e2e = None if args.no_e2e else run_e2e(args, w, inp_cpu, out, lse, stream, world, flops)
 
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops"]            # burst figure: the kernel is timed alone; fp16 dense rate = bf16's
@@ -273,8 +282,7 @@ def main():
                          "mean_launch_ms": mean_launch_ms,
                          "algorithmic_flops_per_launch": flops},
             "gpu_launches": args.steps,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms, "steps": e2e_steps},
+            "e2e": e2e,
             "clocks": clocks.summary()}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

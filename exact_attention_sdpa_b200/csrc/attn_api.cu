@@ -108,14 +108,30 @@ bool encode_qkv_map(CUtensorMap* map, const attn_tensor_t* t) {
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    static int counts[64] = {0};
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
 template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE>
 cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                      cudaStream_t stream) {
     auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE>;
-    constexpr int smem = attn::FwdSmem<D>::kDynBytes;
+    constexpr int smem = attn::Cfg<D>::kDynBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<p.num_units, attn::kThreads, smem, stream>>>(mq, mk, mv, p);
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    // persistent: one CTA per SM (tensor memory and registers allow no more)
+    const int grid = p.num_units < sms ? p.num_units : sms;
+    kern<<<grid, attn::kThreads, smem, stream>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
@@ -224,8 +240,9 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     p.B = static_cast<int>(B);
     p.H = static_cast<int>(H);
     p.N = static_cast<int>(N);
-    p.num_q_tiles = static_cast<int>((N + attn::kBlockM - 1) / attn::kBlockM);
-    const int64_t units = static_cast<int64_t>(p.num_q_tiles) * B * H;
+    p.num_q_pairs = static_cast<int>((N + attn::kRowsPerUnit - 1) / attn::kRowsPerUnit);
+    p.n_kv_tiles = static_cast<int>((N + attn::kBlockN - 1) / attn::kBlockN);
+    const int64_t units = static_cast<int64_t>(p.num_q_pairs) * B * H;
     if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
     p.num_units = static_cast<int>(units);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);

@@ -1,55 +1,74 @@
 // attn_fwd_kernel.cuh -- fused exact attention forward for sm_100a.
 //
-// One CTA owns one 128-row query tile of one (batch, head) and walks its key /
-// value tiles of 128 rows (aiinarabic.com "flash-attention", the per-block
-// order: load a block of Q, K, V on chip, QK^T for the block, softmax of the
-// block, multiply by V, merge with what came before, advance).  The merge is
-// the online softmax of the gist.science FLASHLIGHT summary (Methodology,
-// item 3): a running row maximum m and running sum l, with l and the output
-// accumulator rescaled by e^(m_old - m_new) whenever the maximum grows, so no
-// score or probability tile ever leaves the chip.
+// What it computes (aiinarabic.com "flash-attention", Equation (1), plus the
+// optional additive bias and sigmoid gate of the gated Evoformer variant named
+// in the gist.science FLASHLIGHT summary):
+//     O = softmax(scale * Q K^T [+ bias]) V [* sigmoid(G)],  lse = m + ln(l).
+// How: block by block (aiinarabic.com "flash-attention", the per-block order:
+// load a block of Q, K, V on chip, QK^T of the block, softmax of the block,
+// multiply by V, merge with the previous blocks and move on), merging with the
+// online softmax of the gist.science FLASHLIGHT summary (Methodology, item 3):
+// a running row maximum m and running sum l; whenever m grows, l and the
+// output accumulator are rescaled by 2^(m_old - m_new).  No score or
+// probability tile ever leaves the SM.
 //
-// Roles (warp specialisation):
-//   warps 0-3  softmax: thread t owns query row t of the tile.  It reads its
-//              score row from tensor memory, masks / scales / biases it, updates
-//              m and l, writes the probabilities P (fp16/bf16) back to tensor
-//              memory, rescales its output row when m grew, and finally
-//              normalises, gates and stores O and lse.
-//   warp 4     TMA producer: Q once, then K_j and V_j into a 2-stage ring.
-//   warp 5     MMA issuer (one thread): S_j = Q K_j^T (both operands in shared
-//              memory) into one of two S buffers, and O += P_j V_j with P read
-//              from tensor memory.  S_{j+1} is issued before waiting for P_j so
-//              the next score tile is computed while row softmax runs.
+// Work unit: 256 query rows (two 128-row tiles Q0, Q1) of one (batch, head).
+// The kernel is persistent (one CTA per SM) and walks the units with a static
+// heaviest-first order.  Within a unit the two query tiles ping-pong through
+// the tensor core so that the softmax of one overlaps the MMAs of the other
+// (the B200 counterpart of the matmul / softmax interleave of hamidun.com's
+// FlashAttention-3 article):
+//     tensor core:  S0(j) | PV1(j-1) | S1(j) | PV0(j) | S0(j+1) | PV1(j) | ...
+//     softmax WG0:        [ softmax S0(j) ]          [ softmax S0(j+1) ] ...
+//     softmax WG1:                        [ softmax S1(j) ]          ...
 //
-// Tensor memory (512 columns x 128 lanes, lane = query row):
-//   [0,128)   S buffer 0 (fp32)      [128,256) S buffer 1 (fp32)
-//   [256,320) P buffer 0 (2 x 16-bit per column)
-//   [320,384) P buffer 1             [384,384+d) O accumulator (fp32)
+// Warp roles (16 warps):
+//   WG0 (warps 0-3)   softmax of Q0: thread t owns query row t; reads its score
+//                     row from tensor memory, masks/scales, updates m and l,
+//                     writes P (fp16/bf16) back to tensor memory.
+//   WG1 (warps 4-7)   the same for Q1.
+//   WG2 (warps 8-11)  correction: rescales the O accumulators in tensor memory
+//                     when m grew by more than 2^8 (otherwise the stale maximum
+//                     is kept: the final O/l and lse use the same reference, so
+//                     the result is unchanged), then the epilogue: O/l, gate,
+//                     rounding, stores of O and lse.
+//   warp 12           tcgen05.mma issuer (one thread); allocates tensor memory.
+//   warp 13           TMA producer: Q0, Q1 per unit, K and V tiles into rings.
+//   warps 14-15       idle (they complete warpgroup 3's register hand-back).
 //
-// Every mbarrier wait is bounded; a wait that gives up records a timeout in
-// the device status word, raises a CTA-wide abort flag, and every role then
-// drains what it has in flight and the CTA exits normally.
+// Tensor memory (128 lanes = query rows, 512 columns):
+//   d <= 64:  S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O0 [384,384+d) O1 [384+d, 384+2d)
+//   d = 128:  S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512), P_i in the first 64 columns of S_i
+//             (S_i(j+1) overwrites P_i(j) after PV_i(j), which the single MMA thread issued
+//             earlier; tcgen05.mma operations from one thread execute in issue order).
+//
+// Every mbarrier wait is bounded: a wait that gives up records a timeout in
+// the device status word and raises a CTA-wide abort flag; every role then
+// stops, drains what it has in flight, and the CTA exits without hanging.
 #pragma once
+
+#include <type_traits>
 
 #include "sm100.cuh"
 
 namespace attn {
 
-constexpr int kBlockM = 128;
-constexpr int kBlockN = 128;
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kBlockM = 128;              // rows per query tile (one TMEM lane per row)
+constexpr int kBlockN = 128;              // keys per key/value tile
+constexpr int kRowsPerUnit = 2 * kBlockM;
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColP0 = 256, kColP1 = 320, kColO = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f; // log2 domain: rescale only when m grows by > 2^8
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned long long kDrainLimit = 1ull << 32;
 
 struct FwdParams {
     int B, H, N;
-    int num_q_tiles;
-    int num_units;             // num_q_tiles * B * H
+    int num_q_pairs;           // ceil(N / 256)
+    int num_units;             // num_q_pairs * B * H
+    int n_kv_tiles;            // ceil(N / 128)
     float scale_log2;          // scale * log2(e)
     const void* bias;          // nullable
     int64_t bias_sb, bias_sh, bias_si;   // element strides (bias_sb = 0 when shared over B)
@@ -62,32 +81,66 @@ struct FwdParams {
     unsigned int* status;
 };
 
-struct __align__(8) FwdBarriers {
-    uint64_t q_full;
-    uint64_t k_full[kStages];
-    uint64_t v_full[kStages];
-    uint64_t kv_empty[kStages];
-    uint64_t s_full[2];
-    uint64_t p_full;
-    uint64_t o_done;
+template <int D>
+struct Cfg {
+    static_assert(D == 32 || D == 64 || D == 128, "head dim");
+    // A 128-row tile of D 16-bit elements is stored as D/64 "atoms" of 128 rows
+    // x 128 bytes (128-byte swizzle), or for D = 32 one atom of 128 rows x 64
+    // bytes (64-byte swizzle): exactly the layout TMA writes.
+    static constexpr int kAtomCols = (D >= 64) ? 64 : 32;
+    static constexpr int kNumAtoms = D / kAtomCols;
+    static constexpr int kRowBytes = kAtomCols * 2;
+    static constexpr int kAtomBytes = 128 * kRowBytes;
+    static constexpr int kTileBytes = kNumAtoms * kAtomBytes;     // 128 * D * 2
+    static constexpr uint32_t kLayout = (D >= 64) ? 2u : 4u;      // SW128 : SW64
+    static constexpr uint32_t kSBO = 8 * kRowBytes;               // 8-row group stride
+    static constexpr int kStages = (D == 128) ? 2 : (D == 64 ? 3 : 4);
+    // tensor memory columns
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+    static constexpr uint32_t kColP0 = (D == 128) ? 0 : 256;
+    static constexpr uint32_t kColP1 = (D == 128) ? 128 : 320;
+    static constexpr uint32_t kColO0 = (D == 128) ? 256 : 384;
+    static constexpr uint32_t kColO1 = kColO0 + ((D == 128) ? 128 : D);
+    static_assert(kColO1 + D <= kTmemCols, "tensor memory budget");
+    // shared memory (dynamic, 1024-byte aligned)
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+    static constexpr int kOffV = kOffK + kStages * kTileBytes;
+    static constexpr int kBytes = kOffV + kStages * kTileBytes;
+    static constexpr int kDynBytes = kBytes + 1024;
+    static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <int ST>
+struct __align__(8) FwdShared {
+    uint64_t q_full[2], q_empty[2];
+    uint64_t k_full[ST], k_empty[ST], v_full[ST], v_empty[ST];
+    uint64_t s_full[2];      // MMA -> softmax i: S_i(j) in tensor memory
+    uint64_t pv_ready[2];    // softmax i (P written) + correction (O rescaled) -> MMA
+    uint64_t o_done[2];      // MMA -> correction: PV_i(j) complete
+    uint64_t o_free[2];      // correction -> MMA: epilogue has read O_i
+    uint64_t sm2corr[2];     // softmax i -> correction: alpha (j >= 1) or final m, l
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
+    float alpha[2][kBlockM];
+    float stat_m[2][2][kBlockM];   // [unit parity][tile][row]
+    float stat_l[2][2][kBlockM];
 };
 
 // Bounded wait.  Returns false (and raises the abort flag) if the phase did
 // not complete within `limit` cycles or another role aborted first.
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, FwdBarriers* sb,
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int* abort_flag,
                                            unsigned long long limit, unsigned int* status) {
     const uint32_t a = sm100::smem_u32(bar);
     if (sm100::mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (sm100::mbar_try_wait(a, parity)) return true;
-        if (*reinterpret_cast<volatile int*>(&sb->abort_flag)) return false;
+        if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
         if (static_cast<unsigned long long>(clock64() - t0) > limit) {
             atomicOr(status, kStatusTimeout);
-            *reinterpret_cast<volatile int*>(&sb->abort_flag) = 1;
+            *reinterpret_cast<volatile int*>(abort_flag) = 1;
             return false;
         }
     }
@@ -105,342 +158,464 @@ __device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity, unsi
     }
 }
 
-template <int D>
-struct TileGeom {
-    static_assert(D == 32 || D == 64 || D == 128, "head dim");
-    // a tile of 128 rows x D 16-bit elements is stored as D/64 "atoms" of
-    // 128 rows x 128 bytes (128-byte swizzle), or for D = 32 one atom of
-    // 128 rows x 64 bytes (64-byte swizzle), exactly as TMA writes it.
-    static constexpr int kAtomCols = (D >= 64) ? 64 : 32;       // elements per row per atom
-    static constexpr int kNumAtoms = D / kAtomCols;
-    static constexpr int kRowBytes = kAtomCols * 2;               // 128 or 64
-    static constexpr int kAtomBytes = 128 * kRowBytes;
-    static constexpr int kTileBytes = kNumAtoms * kAtomBytes;     // 128 * D * 2
-    static constexpr uint32_t kLayout = (D >= 64) ? 2u : 4u;      // SW128 : SW64
-    static constexpr uint32_t kSBO = 8 * kRowBytes;               // 8-row group stride
+// Maximum of a 128-entry row with three-input max instructions (two chains).
+__device__ __forceinline__ float row_max(const float (&s)[kBlockN]) {
+    float a0 = s[0], a1 = s[1];
+#pragma unroll
+    for (int c = 2; c + 3 < kBlockN; c += 4) {   // columns 2 .. 125
+        a0 = sm100::max3(a0, s[c], s[c + 1]);
+        a1 = sm100::max3(a1, s[c + 2], s[c + 3]);
+    }
+    return sm100::max3(fmaxf(a0, a1), s[kBlockN - 2], s[kBlockN - 1]);
+}
+
+// One work unit: query rows [q0, q0 + 256) of (b, h); tile i needs key tiles [0, nkv_i).
+struct Unit {
+    int b, h, bh, qp, q0, nkv0, nkv1;
 };
 
-template <int D>
-struct FwdSmem {
-    static constexpr int kTile = TileGeom<D>::kTileBytes;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTile;
-    static constexpr int kOffV = kOffK + kStages * kTile;
-    static constexpr int kBytes = kOffV + kStages * kTile;
-    // pad so that at most one CTA is resident per SM (it allocates all 512 TMEM columns)
-    static constexpr int kDynBytes = (kBytes + 1024 > 120 * 1024) ? (kBytes + 1024) : (120 * 1024);
-};
+template <bool CAUSAL>
+__device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
+    Unit U;
+    const int BH = p.B * p.H;
+    U.qp = p.num_q_pairs - 1 - u / BH;     // heaviest query pairs first
+    U.bh = u % BH;
+    U.b = U.bh / p.H;
+    U.h = U.bh % p.H;
+    U.q0 = U.qp * kRowsPerUnit;
+    if (CAUSAL) {
+        U.nkv0 = min(p.n_kv_tiles, 2 * U.qp + 1);
+        U.nkv1 = min(p.n_kv_tiles, 2 * U.qp + 2);
+    } else {
+        U.nkv0 = U.nkv1 = p.n_kv_tiles;
+    }
+    return U;
+}
 
 template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using namespace sm100;
-    using G = TileGeom<D>;
-    using L = FwdSmem<D>;
+    using C = Cfg<D>;
+    constexpr int ST = C::kStages;
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ FwdBarriers sbar;
+    __shared__ FwdShared<ST> sh;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem + L::kOffQ;
-    uint8_t* sK = smem + L::kOffK;
-    uint8_t* sV = smem + L::kOffV;
+    uint8_t* sQ = smem + C::kOffQ;
+    uint8_t* sK = smem + C::kOffK;
+    uint8_t* sV = smem + C::kOffV;
 
     const int warp = warp_id();
     const int lane = lane_id();
-
-    // work unit: heaviest query tiles first (causal), then (b, h)
-    const int BH = p.B * p.H;
-    const int unit = blockIdx.x;
-    const int qt = p.num_q_tiles - 1 - unit / BH;
-    const int bh = unit % BH;
-    const int b = bh / p.H;
-    const int h = bh % p.H;
-    const int q0 = qt * kBlockM;
-    const int n_kv_all = (p.N + kBlockN - 1) / kBlockN;
-    const int nkv = CAUSAL ? min(n_kv_all, qt + 1) : n_kv_all;
+    const int wg = warp >> 2;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sbar.q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sbar.k_full[s], 1);
-            mbar_init(&sbar.v_full[s], 1);
-            mbar_init(&sbar.kv_empty[s], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sh.q_full[i], 1);
+            mbar_init(&sh.q_empty[i], 1);
+            mbar_init(&sh.s_full[i], 1);
+            mbar_init(&sh.pv_ready[i], 2 * kBlockM);
+            mbar_init(&sh.o_done[i], 1);
+            mbar_init(&sh.o_free[i], kBlockM);
+            mbar_init(&sh.sm2corr[i], kBlockM);
         }
-        mbar_init(&sbar.s_full[0], 1);
-        mbar_init(&sbar.s_full[1], 1);
-        mbar_init(&sbar.p_full, kBlockM);
-        mbar_init(&sbar.o_done, 1);
-        mbar_init(&sbar.drain, 1);
-        sbar.abort_flag = 0;
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.v_full[s], 1);
+            mbar_init(&sh.v_empty[s], 1);
+        }
+        mbar_init(&sh.drain, 1);
+        sh.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 4) {
-        tmem_alloc(&sbar.tmem_base, kTmemCols);
+    if (warp == 12) {
+        tmem_alloc(&sh.tmem_base, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sbar.tmem_base;
+    const uint32_t tmem = sh.tmem_base;
+    int* abort_flag = &sh.abort_flag;
 
-    if (warp == 4) {
-        // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (wg == 3) {
+        regs_dec<80>();
+        if (warp == 13 && lane == 0) {
+            // ============================================================ TMA producer
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
-            mbar_arrive_expect_tx(&sbar.q_full, G::kTileBytes);
-            for (int a = 0; a < G::kNumAtoms; ++a)
-                tma_load_4d(sQ + a * G::kAtomBytes, &tm_q, &sbar.q_full, a * G::kAtomCols, q0, h, b, pol_q);
-            int issued[kStages] = {0, 0};
-            for (int j = 0; j < nkv; ++j) {
-                const int st = j % kStages;
-                if (j >= kStages) {
-                    if (!wait_phase(&sbar.kv_empty[st], ((j / kStages) - 1) & 1, &sbar, p.wait_limit, p.status))
-                        break;
+            uint32_t kc = 0, vc = 0;            // tiles loaded into the K / V rings
+            uint32_t qc[2] = {0, 0};            // Q tiles loaded per slot (one per unit)
+            bool ok = true;
+            auto load_q = [&](int i, const Unit& U) {
+                if (qc[i] > 0) ok = wait_phase(&sh.q_empty[i], (qc[i] - 1) & 1, abort_flag, p.wait_limit, p.status);
+                if (!ok) return;
+                mbar_arrive_expect_tx(&sh.q_full[i], C::kTileBytes);
+                for (int a = 0; a < C::kNumAtoms; ++a)
+                    tma_load_4d(sQ + (i * C::kNumAtoms + a) * C::kAtomBytes, &tm_q, &sh.q_full[i],
+                                a * C::kAtomCols, U.q0 + i * kBlockM, U.h, U.b, pol_q);
+                ++qc[i];
+            };
+            auto load_kv = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, const CUtensorMap* map, uint32_t& cnt,
+                               int j, const Unit& U) {
+                const uint32_t st = cnt % ST;
+                if (cnt >= ST) ok = wait_phase(&empty[st], ((cnt / ST) - 1) & 1, abort_flag, p.wait_limit, p.status);
+                if (!ok) return;
+                mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+                for (int a = 0; a < C::kNumAtoms; ++a)
+                    tma_load_4d(ring + (st * C::kNumAtoms + a) * C::kAtomBytes, map, &full[st], a * C::kAtomCols,
+                                j * kBlockN, U.h, U.b, pol_kv);
+                ++cnt;
+            };
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+                const Unit U = decode_unit<CAUSAL>(u, p);
+                load_q(0, U);
+                if (ok) load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, 0, U);
+                if (ok) load_q(1, U);
+                if (ok) load_kv(sh.v_full, sh.v_empty, sV, &tm_v, vc, 0, U);
+                for (int j = 1; ok && j < U.nkv1; ++j) {
+                    load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, j, U);
+                    if (ok) load_kv(sh.v_full, sh.v_empty, sV, &tm_v, vc, j, U);
                 }
-                uint8_t* dk = sK + st * G::kTileBytes;
-                uint8_t* dv = sV + st * G::kTileBytes;
-                mbar_arrive_expect_tx(&sbar.k_full[st], G::kTileBytes);
-                for (int a = 0; a < G::kNumAtoms; ++a)
-                    tma_load_4d(dk + a * G::kAtomBytes, &tm_k, &sbar.k_full[st], a * G::kAtomCols, j * kBlockN,
-                                h, b, pol_kv);
-                mbar_arrive_expect_tx(&sbar.v_full[st], G::kTileBytes);
-                for (int a = 0; a < G::kNumAtoms; ++a)
-                    tma_load_4d(dv + a * G::kAtomBytes, &tm_v, &sbar.v_full[st], a * G::kAtomCols, j * kBlockN,
-                                h, b, pol_kv);
-                ++issued[st];
             }
-            // drain: every load issued into this CTA's shared memory has landed before exit
-            drain_phase(&sbar.q_full, 0, p.status);
-            for (int st = 0; st < kStages; ++st) {
-                if (issued[st] > 0) {
-                    drain_phase(&sbar.k_full[st], (issued[st] - 1) & 1, p.status);
-                    drain_phase(&sbar.v_full[st], (issued[st] - 1) & 1, p.status);
-                }
+            // drain: every load issued into shared memory lands before the CTA exits
+            for (int i = 0; i < 2; ++i)
+                if (qc[i] > 0) drain_phase(&sh.q_full[i], (qc[i] - 1) & 1, p.status);
+            for (uint32_t s = 0; s < ST; ++s) {
+                if (kc > s) drain_phase(&sh.k_full[s], ((kc - 1 - s) / ST) & 1, p.status);
+                if (vc > s) drain_phase(&sh.v_full[s], ((vc - 1 - s) / ST) & 1, p.status);
             }
-        }
-        __syncwarp();
-    } else if (warp == 5) {
-        // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == 12 && lane == 0) {
+            // ============================================================ MMA issuer
             constexpr uint32_t idesc_s = instr_desc_f16(kBF16, kBlockM, kBlockN, false);
             constexpr uint32_t idesc_o = instr_desc_f16(kBF16, kBlockM, D, true);
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t k_addr = smem_u32(sK);
             const uint32_t v_addr = smem_u32(sV);
-            auto issue_s = [&](int j) {
-                const int st = j % kStages;
-                const uint32_t kb = k_addr + st * G::kTileBytes;
-                const uint32_t dst = tmem + ((j & 1) ? kColS1 : kColS0);
+            constexpr uint32_t kColS[2] = {C::kColS0, C::kColS1};
+            constexpr uint32_t kColP[2] = {C::kColP0, C::kColP1};
+            constexpr uint32_t kColO[2] = {C::kColO0, C::kColO1};
+            // S_i = Q_i K^T: both operands K-major, 16 elements (32 bytes) per step
+            auto issue_s = [&](int i, uint32_t kst) {
+                const uint32_t qb = q_addr + i * C::kTileBytes;
+                const uint32_t kb = k_addr + kst * C::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    // K-major operands: 16 elements (32 bytes) per step inside an atom
-                    const int atom = (kk * 16) / G::kAtomCols;
-                    const uint32_t off = atom * G::kAtomBytes + ((kk * 16) % G::kAtomCols) * 2;
-                    const uint64_t da = smem_desc(q_addr + off, 16, G::kSBO, G::kLayout);
-                    const uint64_t db = smem_desc(kb + off, 16, G::kSBO, G::kLayout);
-                    mma_ss(dst, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk * 16) / C::kAtomCols) * C::kAtomBytes + ((kk * 16) % C::kAtomCols) * 2;
+                    mma_ss(tmem + kColS[i], smem_desc(qb + off, 16, C::kSBO, C::kLayout),
+                           smem_desc(kb + off, 16, C::kSBO, C::kLayout), idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            bool ok = wait_phase(&sbar.q_full, 0, &sbar, p.wait_limit, p.status);
-            if (ok) ok = wait_phase(&sbar.k_full[0], 0, &sbar, p.wait_limit, p.status);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0);
-                mma_commit(&sbar.s_full[0]);
-            }
-            for (int j = 0; ok && j < nkv; ++j) {
-                if (j + 1 < nkv) {
-                    const int st1 = (j + 1) % kStages;
-                    if (!wait_phase(&sbar.k_full[st1], ((j + 1) / kStages) & 1, &sbar, p.wait_limit, p.status))
-                        break;
-                    tc_fence_after();
-                    issue_s(j + 1);
-                    mma_commit(&sbar.s_full[(j + 1) & 1]);
-                }
-                if (!wait_phase(&sbar.p_full, j & 1, &sbar, p.wait_limit, p.status)) break;
-                const int st = j % kStages;
-                if (!wait_phase(&sbar.v_full[st], (j / kStages) & 1, &sbar, p.wait_limit, p.status)) break;
-                tc_fence_after();
-                const uint32_t vb = v_addr + st * G::kTileBytes;
-                const uint32_t pcol = tmem + ((j & 1) ? kColP1 : kColP0);
+            // O_i += P_i V: P from tensor memory, V N(=d)-major in shared memory, 16 keys per step
+            auto issue_pv = [&](int i, uint32_t vst, bool acc) {
+                const uint32_t vb = v_addr + vst * C::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    // V is N(=d)-major: 16 keys per step = 16 rows of the tile
-                    const uint64_t dv = smem_desc(vb + kk * 16 * G::kRowBytes, G::kAtomBytes, G::kSBO, G::kLayout);
-                    mma_ts(tmem + kColO, pcol + kk * 8, dv, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8,
+                           smem_desc(vb + kk * 16 * C::kRowBytes, C::kAtomBytes, C::kSBO, C::kLayout), idesc_o,
+                           (acc || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&sbar.o_done);
-                mma_commit(&sbar.kv_empty[st]);
+            };
+            uint32_t kc = 0, vc = 0, uit = 0;
+            uint32_t pv_cnt[2] = {0, 0};
+            bool ok = true;
+            auto W = [&](uint64_t* bar, uint32_t parity) {
+                if (ok) ok = wait_phase(bar, parity, abort_flag, p.wait_limit, p.status);
+                return ok;
+            };
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
+                const Unit U = decode_unit<CAUSAL>(u, p);
+                // S0(0), S1(0)
+                if (!W(&sh.q_full[0], uit & 1) || !W(&sh.k_full[kc % ST], (kc / ST) & 1)) break;
+                tc_fence_after();
+                issue_s(0, kc % ST);
+                mma_commit(&sh.s_full[0]);
+                if (U.nkv0 == 1) mma_commit(&sh.q_empty[0]);
+                if (!W(&sh.q_full[1], uit & 1)) break;
+                tc_fence_after();
+                issue_s(1, kc % ST);
+                mma_commit(&sh.s_full[1]);
+                mma_commit(&sh.k_empty[kc % ST]);
+                if (U.nkv1 == 1) mma_commit(&sh.q_empty[1]);
+                for (int j = 0; j < U.nkv1; ++j) {
+                    const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
+                    const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
+                    if (j < U.nkv0) {   // PV0(j)
+                        if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
+                        ++pv_cnt[0];
+                        if (j == 0 && uit > 0 && !W(&sh.o_free[0], (uit - 1) & 1)) break;
+                        if (!W(&sh.v_full[vst], vph)) break;
+                        tc_fence_after();
+                        issue_pv(0, vst, j > 0);
+                        mma_commit(&sh.o_done[0]);
+                    }
+                    if (j + 1 < U.nkv0) {   // S0(j+1)
+                        if (!W(&sh.k_full[kst], kph)) break;
+                        tc_fence_after();
+                        issue_s(0, kst);
+                        mma_commit(&sh.s_full[0]);
+                        if (j + 2 == U.nkv0) mma_commit(&sh.q_empty[0]);
+                    }
+                    // PV1(j)
+                    if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
+                    ++pv_cnt[1];
+                    if (j == 0 && uit > 0 && !W(&sh.o_free[1], (uit - 1) & 1)) break;
+                    if (!W(&sh.v_full[vst], vph)) break;
+                    tc_fence_after();
+                    issue_pv(1, vst, j > 0);
+                    mma_commit(&sh.o_done[1]);
+                    mma_commit(&sh.v_empty[vst]);
+                    if (j + 1 < U.nkv1) {   // S1(j+1)
+                        if (!W(&sh.k_full[kst], kph)) break;
+                        tc_fence_after();
+                        issue_s(1, kst);
+                        mma_commit(&sh.s_full[1]);
+                        mma_commit(&sh.k_empty[kst]);
+                        if (j + 2 == U.nkv1) mma_commit(&sh.q_empty[1]);
+                    }
+                }
+                kc += U.nkv1;
+                vc += U.nkv1;
             }
             // drain: all MMAs complete before tensor memory is released
-            mma_commit(&sbar.drain);
-            drain_phase(&sbar.drain, 0, p.status);
+            mma_commit(&sh.drain);
+            drain_phase(&sh.drain, 0, p.status);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------------ softmax / epilogue
-        const int t = threadIdx.x;              // 0..127, the query row within the tile
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const int row = q0 + t;
-        const bool row_ok = row < p.N;
-        float m_run = -INFINITY;                // running max, log2 domain
-        float l_run = 0.f;                      // running sum
+    } else if (wg < 2) {
+        // ================================================================ softmax of tile i = wg
+        regs_inc<176>();
+        const int i = wg;
+        const int t = threadIdx.x & 127;          // row within the tile
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t col_s = i ? Cfg<D>::kColS1 : Cfg<D>::kColS0;
+        const uint32_t col_p = i ? Cfg<D>::kColP1 : Cfg<D>::kColP0;
+        const float scale_log2 = p.scale_log2;
+        const bool fast = !HAS_BIAS && scale_log2 > 0.f;   // max over raw scores, fused scale
+        uint32_t s_cnt = 0, uit = 0;
         bool ok = true;
-        const T* bias_row = nullptr;
-        if constexpr (HAS_BIAS) {
-            bias_row = reinterpret_cast<const T*>(p.bias) + b * p.bias_sb + h * p.bias_sh +
-                       static_cast<int64_t>(row_ok ? row : 0) * p.bias_si;
-        }
-
-        for (int j = 0; j < nkv; ++j) {
-            const int sbuf = j & 1;
-            ok = wait_phase(&sbar.s_full[sbuf], (j >> 1) & 1, &sbar, p.wait_limit, p.status);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-
-            float s[kBlockN];
-            {
-                uint32_t r[32];
-#pragma unroll
-                for (int c = 0; c < kBlockN / 32; ++c) {
-                    tmem_ld32(tmem + lane_off + (sbuf ? kColS1 : kColS0) + c * 32, r);
-                    tmem_wait_ld(r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-                }
-            }
-            const int kv0 = j * kBlockN;
-            const bool need_mask = (kv0 + kBlockN > p.N) || (CAUSAL && j == qt);
-            float mx = m_run;
-#pragma unroll
-            for (int c = 0; c < kBlockN; c += 8) {
-                float bv[8];
-                if constexpr (HAS_BIAS) {
-                    if (row_ok && kv0 + c + 8 <= p.N) {
-                        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
-                        const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) bv[i] = to_f32<T>(e[i]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            bv[i] = (row_ok && kv0 + c + i < p.N) ? to_f32<T>(bias_row[kv0 + c + i]) : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float x = s[c + i] * p.scale_log2;
-                    if constexpr (HAS_BIAS) x = fmaf(bv[i], kLog2e, x);
-                    if (need_mask) {
-                        const int key = kv0 + c + i;
-                        if (key >= p.N || (CAUSAL && key > row)) x = -INFINITY;
-                    }
-                    s[c + i] = x;
-                    mx = fmaxf(mx, x);
-                }
-            }
-            const float alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mx);
-            const float m_use = (mx == -INFINITY) ? 0.f : mx;
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < kBlockN; ++c) {
-                const float e = ex2_approx(s[c] - m_use);
-                s[c] = e;
-                sum += e;
-            }
-            l_run = fmaf(l_run, alpha, sum);
-            m_run = mx;
-
-            // O_{j-1} must be complete before rescaling O (and before P_{j} overwrites P_{j-2}'s buffer)
-            if (j > 0) {
-                ok = wait_phase(&sbar.o_done, (j - 1) & 1, &sbar, p.wait_limit, p.status);
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
+            const Unit U = decode_unit<CAUSAL>(u, p);
+            const int nkv = i ? U.nkv1 : U.nkv0;
+            const int row = U.q0 + i * kBlockM + t;
+            const int diag = 2 * U.qp + i;          // the key tile holding this tile's diagonal
+            const T* bias_row = nullptr;
+            if constexpr (HAS_BIAS)
+                bias_row = reinterpret_cast<const T*>(p.bias) + U.b * p.bias_sb + U.h * p.bias_sh +
+                           static_cast<int64_t>(row < p.N ? row : 0) * p.bias_si;
+            float m_ref = -INFINITY;                // reference maximum (log2 domain)
+            float l = 0.f;
+            for (int j = 0; j < nkv; ++j) {
+                ok = wait_phase(&sh.s_full[i], s_cnt & 1, abort_flag, p.wait_limit, p.status);
+                ++s_cnt;
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
+                float s[kBlockN];
+                {
+                    uint32_t r[kBlockN];
+#pragma unroll
+                    for (int c = 0; c < kBlockN / 32; ++c)
+                        tmem_ld32(tmem + lane_off + col_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+                    tmem_wait_ld128(r);
+#pragma unroll
+                    for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(r[c]);
+                }
+                const int kv0 = j * kBlockN;
+                const bool need_mask = (kv0 + kBlockN > p.N) || (CAUSAL && j == diag);
+                float m_tile;   // tile maximum, log2 domain
+                if (fast) {
+                    if (need_mask) {
+                        const int lim = CAUSAL ? min(p.N - kv0, row - kv0 + 1) : (p.N - kv0);
+#pragma unroll
+                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+                    }
+                    m_tile = row_max(s) * scale_log2;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kBlockN; c += 8) {
+                        float bv[8];
+                        if constexpr (HAS_BIAS) {
+                            if (row < p.N && kv0 + c + 8 <= p.N) {
+                                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
+                                const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) bv[q] = to_f32<T>(e[q]);
+                            } else {
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    bv[q] = (row < p.N && kv0 + c + q < p.N) ? to_f32<T>(bias_row[kv0 + c + q]) : 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float x = s[c + q] * scale_log2;
+                            if constexpr (HAS_BIAS) x = fmaf(bv[q], kLog2e, x);
+                            s[c + q] = x;
+                        }
+                    }
+                    if (need_mask) {
+                        const int lim = CAUSAL ? min(p.N - kv0, row - kv0 + 1) : (p.N - kv0);
+#pragma unroll
+                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+                    }
+                    m_tile = row_max(s);
+                }
+                // reference maximum: move it only when the row maximum grew by more than the threshold
+                float m_new = m_ref, alpha = 1.f;
+                if (m_ref == -INFINITY) {
+                    m_new = m_tile;
+                    alpha = 0.f;
+                } else if (m_tile > m_ref + kRescaleThreshold) {
+                    m_new = m_tile;
+                    alpha = ex2_approx(m_ref - m_new);
+                }
+                if (j > 0) {
+                    sh.alpha[i][t] = alpha;
+                    mbar_arrive(&sh.sm2corr[i]);
+                }
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                float sum0 = 0.f, sum1 = 0.f;
+                if (fast) {
+                    const float neg = -m_use;
+#pragma unroll
+                    for (int c = 0; c < kBlockN; c += 2) {
+                        float x0, x1;
+                        ffma2(x0, x1, s[c], s[c + 1], scale_log2, scale_log2, neg, neg);
+                        s[c] = ex2_approx(x0);
+                        s[c + 1] = ex2_approx(x1);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kBlockN; c += 2) {
+                        float x0, x1;
+                        fadd2(x0, x1, s[c], s[c + 1], -m_use, -m_use);
+                        s[c] = ex2_approx(x0);
+                        s[c + 1] = ex2_approx(x1);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < kBlockN; c += 2) fadd2(sum0, sum1, sum0, sum1, s[c], s[c + 1]);
+                l = fmaf(l, alpha, sum0 + sum1);
+                m_ref = m_new;
+                {
+                    uint32_t pk[64];
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) pk[c] = pack2<T>(s[2 * c], s[2 * c + 1]);
+                    tmem_st64(tmem + lane_off + col_p, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sh.pv_ready[i]);
             }
-            {
-                uint32_t pk[32];
+            if (!ok) break;
+            sh.stat_m[uit & 1][i][t] = m_ref;
+            sh.stat_l[uit & 1][i][t] = l;
+            mbar_arrive(&sh.sm2corr[i]);
+        }
+    } else {
+        // ================================================================ correction + epilogue
+        regs_dec<80>();
+        const int t = threadIdx.x & 127;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        constexpr uint32_t kColO[2] = {Cfg<D>::kColO0, Cfg<D>::kColO1};
+        uint32_t c_cnt[2] = {0, 0}, od_cnt[2] = {0, 0}, uit = 0;
+        bool ok = true;
+        auto WS = [&](uint64_t* bar, uint32_t& cnt) {
+            if (ok) ok = wait_phase(bar, cnt & 1, abort_flag, p.wait_limit, p.status);
+            ++cnt;
+            ok = __all_sync(0xffffffffu, ok);
+            return ok;
+        };
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
+            const Unit U = decode_unit<CAUSAL>(u, p);
+            for (int j = 0; ok && j < U.nkv1; ++j) {
+                for (int i = 0; i < 2; ++i) {
+                    if (j >= (i ? U.nkv1 : U.nkv0)) continue;
+                    if (j > 0) {
+                        if (!WS(&sh.sm2corr[i], c_cnt[i])) break;
+                        const float alpha = sh.alpha[i][t];
+                        if (!WS(&sh.o_done[i], od_cnt[i])) break;   // PV_i(j-1) complete
+                        tc_fence_after();
+                        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                            uint32_t r[32];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                            for (int c = 0; c < D / 32; ++c) {
+                                tmem_ld32(tmem + lane_off + kColO[i] + c * 32, r);
+                                tmem_wait_ld(r);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pk[i] = pack2<T>(s[half * 64 + 2 * i], s[half * 64 + 2 * i + 1]);
-                    tmem_st32(tmem + lane_off + (sbuf ? kColP1 : kColP0) + half * 32, pk);
+                                for (int q = 0; q < 32; q += 2) {
+                                    float x0, x1;
+                                    fmul2(x0, x1, __uint_as_float(r[q]), __uint_as_float(r[q + 1]), alpha, alpha);
+                                    r[q] = __float_as_uint(x0);
+                                    r[q + 1] = __float_as_uint(x1);
+                                }
+                                tmem_st32(tmem + lane_off + kColO[i] + c * 32, r);
+                            }
+                            tmem_wait_st();
+                        }
+                        tc_fence_before();
+                    }
+                    mbar_arrive(&sh.pv_ready[i]);
                 }
             }
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (!ok) break;
+            // epilogue: O = O_acc / l (* sigmoid(G)), lse = (m + log2 l) * ln 2
+            for (int i = 0; i < 2; ++i) {
+                if (!WS(&sh.sm2corr[i], c_cnt[i])) break;      // final m, l
+                if (!WS(&sh.o_done[i], od_cnt[i])) break;      // last PV_i complete
+                tc_fence_after();
+                const float m = sh.stat_m[uit & 1][i][t];
+                const float l = sh.stat_l[uit & 1][i][t];
+                const int row = U.q0 + i * kBlockM + t;
+                const bool row_ok = row < p.N;
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                T* orow = reinterpret_cast<T*>(p.out) + U.b * p.out_sb + U.h * p.out_sh +
+                          static_cast<int64_t>(row_ok ? row : 0) * p.out_si;
+                const T* grow = nullptr;
+                if constexpr (HAS_GATE)
+                    grow = reinterpret_cast<const T*>(p.gate) + U.b * p.gate_sb + U.h * p.gate_sh +
+                           static_cast<int64_t>(row_ok ? row : 0) * p.gate_si;
                 uint32_t r[32];
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32(tmem + lane_off + kColO + c * 32, r);
+                    tmem_ld32(tmem + lane_off + kColO[i] + c * 32, r);
                     tmem_wait_ld(r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(tmem + lane_off + kColO + c * 32, r);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sbar.p_full);
-        }
-
-        if (ok) {
-            ok = wait_phase(&sbar.o_done, (nkv - 1) & 1, &sbar, p.wait_limit, p.status);
-            ok = __all_sync(0xffffffffu, ok);
-        }
-        if (ok) {
-            tc_fence_after();
-            const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-            T* orow = reinterpret_cast<T*>(p.out) + b * p.out_sb + h * p.out_sh +
-                      static_cast<int64_t>(row_ok ? row : 0) * p.out_si;
-            const T* grow = nullptr;
-            if constexpr (HAS_GATE)
-                grow = reinterpret_cast<const T*>(p.gate) + b * p.gate_sb + h * p.gate_sh +
-                       static_cast<int64_t>(row_ok ? row : 0) * p.gate_si;
-            uint32_t r[32];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                tmem_ld32(tmem + lane_off + kColO + c * 32, r);
-                tmem_wait_ld(r);
-                float o[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]) * inv_l;
-                if constexpr (HAS_GATE) {
                     if (row_ok) {
 #pragma unroll
                         for (int v8 = 0; v8 < 4; ++v8) {
-                            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(grow + c * 32 + v8 * 8));
-                            const T* e = reinterpret_cast<const T*>(&raw);
+                            float o[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const float g = to_f32<T>(e[i]);
-                                o[v8 * 8 + i] *= 1.f / (1.f + ex2_approx(-g * kLog2e));
+                            for (int q = 0; q < 8; ++q) o[q] = __uint_as_float(r[v8 * 8 + q]) * inv_l;
+                            if constexpr (HAS_GATE) {
+                                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(grow + c * 32 + v8 * 8));
+                                const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    o[q] *= 1.f / (1.f + ex2_approx(-to_f32<T>(e[q]) * kLog2e));
                             }
+                            uint4 w;
+                            w.x = pack2<T>(o[0], o[1]);
+                            w.y = pack2<T>(o[2], o[3]);
+                            w.z = pack2<T>(o[4], o[5]);
+                            w.w = pack2<T>(o[6], o[7]);
+                            *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = w;
                         }
                     }
                 }
-                if (row_ok) {
-#pragma unroll
-                    for (int v8 = 0; v8 < 4; ++v8) {
-                        uint4 w;
-                        w.x = pack2<T>(o[v8 * 8 + 0], o[v8 * 8 + 1]);
-                        w.y = pack2<T>(o[v8 * 8 + 2], o[v8 * 8 + 3]);
-                        w.z = pack2<T>(o[v8 * 8 + 4], o[v8 * 8 + 5]);
-                        w.w = pack2<T>(o[v8 * 8 + 6], o[v8 * 8 + 7]);
-                        *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = w;
-                    }
-                }
-            }
-            if (p.lse != nullptr && row_ok) {
-                const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * kLn2 : -INFINITY;
-                p.lse[static_cast<int64_t>(bh) * p.N + row] = lse;
+                if (p.lse != nullptr && row_ok)
+                    p.lse[static_cast<int64_t>(U.bh) * p.N + row] =
+                        (l > 0.f) ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
+                tc_fence_before();
+                mbar_arrive(&sh.o_free[i]);
             }
         }
     }
@@ -448,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
