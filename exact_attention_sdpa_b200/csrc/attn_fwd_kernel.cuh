@@ -96,6 +96,9 @@ struct Cfg {
     static constexpr uint32_t kSBO = 8 * kRowBytes;               // 8-row group stride
     static constexpr int kStages = (D == 128) ? 2 : (D == 64 ? 3 : 4);
     // tensor memory columns
+    // d <= 64: P has columns of its own, so S_i(j+1) may be computed while the
+    // softmax of S_i(j) runs; d = 128: P lives inside S_i (no room otherwise).
+    static constexpr bool kSeparateP = (D <= 64);
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColP0 = (D == 128) ? 0 : 256;
     static constexpr uint32_t kColP1 = (D == 128) ? 128 : 320;
@@ -116,14 +119,16 @@ struct __align__(8) FwdShared {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[ST], k_empty[ST], v_full[ST], v_empty[ST];
     uint64_t s_full[2];      // MMA -> softmax i: S_i(j) in tensor memory
+    uint64_t s_free[2];      // softmax i -> MMA: S_i(j) read into registers (d <= 64 only)
     uint64_t pv_ready[2];    // softmax i (P written) + correction (O rescaled) -> MMA
     uint64_t o_done[2];      // MMA -> correction: PV_i(j) complete
     uint64_t o_free[2];      // correction -> MMA: epilogue has read O_i
-    uint64_t sm2corr[2];     // softmax i -> correction: alpha (j >= 1) or final m, l
+    uint64_t sm2corr[2];     // softmax i -> correction: alpha(j), j >= 1
+    uint64_t stats_full[2];  // softmax i -> correction: final m, l of the unit
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
-    float alpha[2][kBlockM];
+    float alpha[2][2][kBlockM];    // [iteration parity][tile][row]
     float stat_m[2][2][kBlockM];   // [unit parity][tile][row]
     float stat_l[2][2][kBlockM];
 };
@@ -158,15 +163,44 @@ __device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity, unsi
     }
 }
 
-// Maximum of a 128-entry row with three-input max instructions (two chains).
+// Maximum of a 128-entry row: eight independent chains of three-input max
+// instructions (dependency depth 10 instead of 43), then a small tree.
 __device__ __forceinline__ float row_max(const float (&s)[kBlockN]) {
-    float a0 = s[0], a1 = s[1];
+    float m[8];
 #pragma unroll
-    for (int c = 2; c + 3 < kBlockN; c += 4) {   // columns 2 .. 125
-        a0 = sm100::max3(a0, s[c], s[c + 1]);
-        a1 = sm100::max3(a1, s[c + 2], s[c + 3]);
+    for (int q = 0; q < 8; ++q) {
+        float a = fmaxf(s[16 * q], s[16 * q + 1]);
+#pragma unroll
+        for (int c = 2; c < 16; c += 2) a = sm100::max3(a, s[16 * q + c], s[16 * q + c + 1]);
+        m[q] = a;
     }
-    return sm100::max3(fmaxf(a0, a1), s[kBlockN - 2], s[kBlockN - 1]);
+    return sm100::max3(sm100::max3(m[0], m[1], m[2]), sm100::max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// 2^x for two lanes on the FMA and integer pipes instead of the MUFU unit.
+// Range reduction in the style of Cody and Waite: n = floor(x) by a
+// round-toward-minus-infinity add of 1.5 * 2^23 (n then sits in the low
+// mantissa bits of t), f = x - n in [0, 1); 2^f by a cubic whose
+// coefficients we fitted for minimum relative error on [0, 1) (max relative
+// error 7.5e-5, below the half-ulp of the fp16/bf16 P it feeds); finally n is
+// added to the exponent field.  Inputs below -126 are clamped there, which
+// yields at most a denormal that the fp16 rounding and the flushed row sum
+// discard.
+__device__ __forceinline__ void ex2_emu2(float& y0, float& y1, float x0, float x1) {
+    constexpr float kShift = 12582912.f;                     // 1.5 * 2^23
+    constexpr float c0 = 0.9999251814280168f, c1 = 0.6958336953498905f;
+    constexpr float c2 = 0.2260672333620784f, c3 = 0.07802422535748339f;
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float t0, t1, r0, r1, f0, f1, p0, p1;
+    sm100::fadd2_rm(t0, t1, x0, x1, kShift, kShift);        // kShift + floor(x)
+    sm100::fadd2(r0, r1, t0, t1, -kShift, -kShift);          // floor(x), exact
+    sm100::fsub2(f0, f1, x0, x1, r0, r1);                    // f in [0, 1)
+    sm100::ffma2(p0, p1, f0, f1, c3, c3, c2, c2);
+    sm100::ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    sm100::ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // One work unit: query rows [q0, q0 + 256) of (b, h); tile i needs key tiles [0, nkv_i).
@@ -217,10 +251,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh.q_full[i], 1);
             mbar_init(&sh.q_empty[i], 1);
             mbar_init(&sh.s_full[i], 1);
+            mbar_init(&sh.s_free[i], kBlockM);
             mbar_init(&sh.pv_ready[i], 2 * kBlockM);
             mbar_init(&sh.o_done[i], 1);
             mbar_init(&sh.o_free[i], kBlockM);
             mbar_init(&sh.sm2corr[i], kBlockM);
+            mbar_init(&sh.stats_full[i], kBlockM);
         }
         for (int s = 0; s < ST; ++s) {
             mbar_init(&sh.k_full[s], 1);
@@ -245,34 +281,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (wg == 3) {
         regs_dec<80>();
-        if (warp == 13 && lane == 0) {
+        if (warp == 13) {
             // ============================================================ TMA producer
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
+            // The whole warp runs this loop (uniform control flow); one elected lane issues.
+            if (elect_one()) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+            }
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
             uint32_t kc = 0, vc = 0;            // tiles loaded into the K / V rings
             uint32_t qc[2] = {0, 0};            // Q tiles loaded per slot (one per unit)
             bool ok = true;
+            auto WU = [&](uint64_t* bar, uint32_t parity) {
+                if (ok) ok = wait_phase(bar, parity, abort_flag, p.wait_limit, p.status);
+                ok = __all_sync(0xffffffffu, ok);
+                return ok;
+            };
             auto load_q = [&](int i, const Unit& U) {
-                if (qc[i] > 0) ok = wait_phase(&sh.q_empty[i], (qc[i] - 1) & 1, abort_flag, p.wait_limit, p.status);
-                if (!ok) return;
-                mbar_arrive_expect_tx(&sh.q_full[i], C::kTileBytes);
-                for (int a = 0; a < C::kNumAtoms; ++a)
-                    tma_load_4d(sQ + (i * C::kNumAtoms + a) * C::kAtomBytes, &tm_q, &sh.q_full[i],
-                                a * C::kAtomCols, U.q0 + i * kBlockM, U.h, U.b, pol_q);
+                if (qc[i] > 0 && !WU(&sh.q_empty[i], (qc[i] - 1) & 1)) return;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&sh.q_full[i], C::kTileBytes);
+                    for (int a = 0; a < C::kNumAtoms; ++a)
+                        tma_load_4d(sQ + (i * C::kNumAtoms + a) * C::kAtomBytes, &tm_q, &sh.q_full[i],
+                                    a * C::kAtomCols, U.q0 + i * kBlockM, U.h, U.b, pol_q);
+                }
+                __syncwarp();
                 ++qc[i];
             };
             auto load_kv = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, const CUtensorMap* map, uint32_t& cnt,
                                int j, const Unit& U) {
                 const uint32_t st = cnt % ST;
-                if (cnt >= ST) ok = wait_phase(&empty[st], ((cnt / ST) - 1) & 1, abort_flag, p.wait_limit, p.status);
-                if (!ok) return;
-                mbar_arrive_expect_tx(&full[st], C::kTileBytes);
-                for (int a = 0; a < C::kNumAtoms; ++a)
-                    tma_load_4d(ring + (st * C::kNumAtoms + a) * C::kAtomBytes, map, &full[st], a * C::kAtomCols,
-                                j * kBlockN, U.h, U.b, pol_kv);
+                if (cnt >= ST && !WU(&empty[st], ((cnt / ST) - 1) & 1)) return;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+                    for (int a = 0; a < C::kNumAtoms; ++a)
+                        tma_load_4d(ring + (st * C::kNumAtoms + a) * C::kAtomBytes, map, &full[st],
+                                    a * C::kAtomCols, j * kBlockN, U.h, U.b, pol_kv);
+                }
+                __syncwarp();
                 ++cnt;
             };
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
@@ -293,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kc > s) drain_phase(&sh.k_full[s], ((kc - 1 - s) / ST) & 1, p.status);
                 if (vc > s) drain_phase(&sh.v_full[s], ((vc - 1 - s) / ST) & 1, p.status);
             }
-        } else if (warp == 12 && lane == 0) {
+        } else if (warp == 12) {
             // ============================================================ MMA issuer
             constexpr uint32_t idesc_s = instr_desc_f16(kBF16, kBlockM, kBlockN, false);
             constexpr uint32_t idesc_o = instr_desc_f16(kBF16, kBlockM, D, true);
@@ -303,32 +351,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kColS[2] = {C::kColS0, C::kColS1};
             constexpr uint32_t kColP[2] = {C::kColP0, C::kColP1};
             constexpr uint32_t kColO[2] = {C::kColO0, C::kColO1};
+            // Descriptors are affine in the start address (bits [0,14) hold address / 16 and
+            // shared addresses stay below 256 KB), so each step adds a constant to a base.
+            const uint64_t dq = smem_desc(q_addr, 16, C::kSBO, C::kLayout);
+            const uint64_t dk = smem_desc(k_addr, 16, C::kSBO, C::kLayout);
+            const uint64_t dv = smem_desc(v_addr, C::kAtomBytes, C::kSBO, C::kLayout);
             // S_i = Q_i K^T: both operands K-major, 16 elements (32 bytes) per step
             auto issue_s = [&](int i, uint32_t kst) {
-                const uint32_t qb = q_addr + i * C::kTileBytes;
-                const uint32_t kb = k_addr + kst * C::kTileBytes;
+                const uint64_t qb = dq + ((i * C::kTileBytes) >> 4);
+                const uint64_t kb = dk + ((kst * C::kTileBytes) >> 4);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk * 16) / C::kAtomCols) * C::kAtomBytes + ((kk * 16) % C::kAtomCols) * 2;
-                    mma_ss(tmem + kColS[i], smem_desc(qb + off, 16, C::kSBO, C::kLayout),
-                           smem_desc(kb + off, 16, C::kSBO, C::kLayout), idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off =
+                            (((kk * 16) / C::kAtomCols) * C::kAtomBytes + ((kk * 16) % C::kAtomCols) * 2) >> 4;
+                        mma_ss(tmem + kColS[i], qb + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
+                    }
                 }
+                __syncwarp();
             };
             // O_i += P_i V: P from tensor memory, V N(=d)-major in shared memory, 16 keys per step
             auto issue_pv = [&](int i, uint32_t vst, bool acc) {
-                const uint32_t vb = v_addr + vst * C::kTileBytes;
+                const uint64_t vb = dv + ((vst * C::kTileBytes) >> 4);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8,
-                           smem_desc(vb + kk * 16 * C::kRowBytes, C::kAtomBytes, C::kSBO, C::kLayout), idesc_o,
-                           (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBlockN / 16; ++kk)
+                        mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8, vb + ((kk * 16 * C::kRowBytes) >> 4),
+                               idesc_o, (acc || kk > 0) ? 1u : 0u);
                 }
+                __syncwarp();
+            };
+            auto commit = [&](uint64_t* bar) {
+                if (elect_one()) mma_commit(bar);
+                __syncwarp();
             };
             uint32_t kc = 0, vc = 0, uit = 0;
-            uint32_t pv_cnt[2] = {0, 0};
+            uint32_t pv_cnt[2] = {0, 0}, sf_cnt[2] = {0, 0};
             bool ok = true;
             auto W = [&](uint64_t* bar, uint32_t parity) {
                 if (ok) ok = wait_phase(bar, parity, abort_flag, p.wait_limit, p.status);
+                ok = __all_sync(0xffffffffu, ok);
                 return ok;
             };
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
@@ -337,17 +399,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!W(&sh.q_full[0], uit & 1) || !W(&sh.k_full[kc % ST], (kc / ST) & 1)) break;
                 tc_fence_after();
                 issue_s(0, kc % ST);
-                mma_commit(&sh.s_full[0]);
-                if (U.nkv0 == 1) mma_commit(&sh.q_empty[0]);
+                commit(&sh.s_full[0]);
+                if (U.nkv0 == 1) commit(&sh.q_empty[0]);
                 if (!W(&sh.q_full[1], uit & 1)) break;
                 tc_fence_after();
                 issue_s(1, kc % ST);
-                mma_commit(&sh.s_full[1]);
-                mma_commit(&sh.k_empty[kc % ST]);
-                if (U.nkv1 == 1) mma_commit(&sh.q_empty[1]);
+                commit(&sh.s_full[1]);
+                commit(&sh.k_empty[kc % ST]);
+                if (U.nkv1 == 1) commit(&sh.q_empty[1]);
                 for (int j = 0; j < U.nkv1; ++j) {
                     const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
                     const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
+                    if constexpr (C::kSeparateP) {
+                        // S0(j+1), S1(j+1) as soon as the softmax has read S(j); then PV0(j), PV1(j)
+                        if (j + 1 < U.nkv0) {
+                            if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
+                            ++sf_cnt[0];
+                            if (!W(&sh.k_full[kst], kph)) break;
+                            tc_fence_after();
+                            issue_s(0, kst);
+                            commit(&sh.s_full[0]);
+                            if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
+                        }
+                        if (j + 1 < U.nkv1) {
+                            if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
+                            ++sf_cnt[1];
+                            if (!W(&sh.k_full[kst], kph)) break;
+                            tc_fence_after();
+                            issue_s(1, kst);
+                            commit(&sh.s_full[1]);
+                            commit(&sh.k_empty[kst]);
+                            if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
+                        }
+                        if (j < U.nkv0) {
+                            if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
+                            ++pv_cnt[0];
+                            if (j == 0 && uit > 0 && !W(&sh.o_free[0], (uit - 1) & 1)) break;
+                            if (!W(&sh.v_full[vst], vph)) break;
+                            tc_fence_after();
+                            issue_pv(0, vst, j > 0);
+                            commit(&sh.o_done[0]);
+                        }
+                        if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
+                        ++pv_cnt[1];
+                        if (j == 0 && uit > 0 && !W(&sh.o_free[1], (uit - 1) & 1)) break;
+                        if (!W(&sh.v_full[vst], vph)) break;
+                        tc_fence_after();
+                        issue_pv(1, vst, j > 0);
+                        commit(&sh.o_done[1]);
+                        commit(&sh.v_empty[vst]);
+                        continue;
+                    }
                     if (j < U.nkv0) {   // PV0(j)
                         if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
                         ++pv_cnt[0];
@@ -355,14 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!W(&sh.v_full[vst], vph)) break;
                         tc_fence_after();
                         issue_pv(0, vst, j > 0);
-                        mma_commit(&sh.o_done[0]);
+                        commit(&sh.o_done[0]);
                     }
                     if (j + 1 < U.nkv0) {   // S0(j+1)
                         if (!W(&sh.k_full[kst], kph)) break;
                         tc_fence_after();
                         issue_s(0, kst);
-                        mma_commit(&sh.s_full[0]);
-                        if (j + 2 == U.nkv0) mma_commit(&sh.q_empty[0]);
+                        commit(&sh.s_full[0]);
+                        if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
                     }
                     // PV1(j)
                     if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
@@ -371,22 +473,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!W(&sh.v_full[vst], vph)) break;
                     tc_fence_after();
                     issue_pv(1, vst, j > 0);
-                    mma_commit(&sh.o_done[1]);
-                    mma_commit(&sh.v_empty[vst]);
+                    commit(&sh.o_done[1]);
+                    commit(&sh.v_empty[vst]);
                     if (j + 1 < U.nkv1) {   // S1(j+1)
                         if (!W(&sh.k_full[kst], kph)) break;
                         tc_fence_after();
                         issue_s(1, kst);
-                        mma_commit(&sh.s_full[1]);
-                        mma_commit(&sh.k_empty[kst]);
-                        if (j + 2 == U.nkv1) mma_commit(&sh.q_empty[1]);
+                        commit(&sh.s_full[1]);
+                        commit(&sh.k_empty[kst]);
+                        if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
                     }
                 }
                 kc += U.nkv1;
                 vc += U.nkv1;
             }
             // drain: all MMAs complete before tensor memory is released
-            mma_commit(&sh.drain);
+            commit(&sh.drain);
             drain_phase(&sh.drain, 0, p.status);
         }
         __syncwarp();
@@ -400,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t col_p = i ? Cfg<D>::kColP1 : Cfg<D>::kColP0;
         const float scale_log2 = p.scale_log2;
         const bool fast = !HAS_BIAS && scale_log2 > 0.f;   // max over raw scores, fused scale
-        uint32_t s_cnt = 0, uit = 0;
+        uint32_t s_cnt = 0, od_cnt = 0, uit = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
             const Unit U = decode_unit<CAUSAL>(u, p);
@@ -428,6 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld128(r);
 #pragma unroll
                     for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(r[c]);
+                }
+                if constexpr (Cfg<D>::kSeparateP) {
+                    if (j + 1 < nkv) {      // S_i may now be overwritten by S_i(j+1)
+                        tc_fence_before();
+                        mbar_arrive(&sh.s_free[i]);
+                    }
                 }
                 const int kv0 = j * kBlockN;
                 const bool need_mask = (kv0 + kBlockN > p.N) || (CAUSAL && j == diag);
@@ -478,48 +586,66 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_new = m_tile;
                     alpha = ex2_approx(m_ref - m_new);
                 }
-                if (j > 0) {
-                    sh.alpha[i][t] = alpha;
+                if (!Cfg<D>::kSeparateP && j > 0) {
+                    // S_i(j) was issued after PV_i(j-1), so the correction has consumed alpha(j-1)
+                    sh.alpha[j & 1][i][t] = alpha;
                     mbar_arrive(&sh.sm2corr[i]);
                 }
                 const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                float sum0 = 0.f, sum1 = 0.f;
-                if (fast) {
-                    const float neg = -m_use;
+                // p = 2^(x - m): x = s * scale_log2 on the fast path (s raw), x = s otherwise.
+                // One pair in three goes through the FMA-pipe exponential so that the
+                // MUFU unit (16 lanes per clock per SM) is not the only exp resource.
+                const float xa = fast ? scale_log2 : 1.f;
+                const float xb = -m_use;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < kBlockN; c += 2) {
-                        float x0, x1;
-                        ffma2(x0, x1, s[c], s[c + 1], scale_log2, scale_log2, neg, neg);
-                        s[c] = ex2_approx(x0);
-                        s[c + 1] = ex2_approx(x1);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int q2 = 0; q2 < 32; ++q2) {
+                        const int pp = half * 32 + q2;
+                        float x0, x1, e0, e1;
+                        ffma2(x0, x1, s[2 * pp], s[2 * pp + 1], xa, xa, xb, xb);
+                        if (pp % 3 == 2) {
+                            ex2_emu2(e0, e1, x0, x1);
+                        } else {
+                            e0 = ex2_approx(x0);
+                            e1 = ex2_approx(x1);
+                        }
+                        const int q = (pp & 3) * 2;
+                        fadd2_ftz(acc[q], acc[q + 1], acc[q], acc[q + 1], e0, e1);
+                        pk[q2] = pack2<T>(e0, e1);
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < kBlockN; c += 2) {
-                        float x0, x1;
-                        fadd2(x0, x1, s[c], s[c + 1], -m_use, -m_use);
-                        s[c] = ex2_approx(x0);
-                        s[c + 1] = ex2_approx(x1);
+                    if constexpr (Cfg<D>::kSeparateP) {
+                        // P_i(j) overwrites P_i(j-1): PV_i(j-1) must have completed.  Its
+                        // completion also means the correction consumed alpha(j-1), so alpha(j)
+                        // is published only now (its barrier never runs two phases ahead).
+                        if (half == 0 && j > 0) {
+                            ok = wait_phase(&sh.o_done[i], od_cnt & 1, abort_flag, p.wait_limit, p.status);
+                            ++od_cnt;
+                            ok = __all_sync(0xffffffffu, ok);
+                            if (ok) {
+                                tc_fence_after();
+                                sh.alpha[j & 1][i][t] = alpha;
+                                mbar_arrive(&sh.sm2corr[i]);
+                            }
+                        }
                     }
-                }
-#pragma unroll
-                for (int c = 0; c < kBlockN; c += 2) fadd2(sum0, sum1, sum0, sum1, s[c], s[c + 1]);
-                l = fmaf(l, alpha, sum0 + sum1);
-                m_ref = m_new;
-                {
-                    uint32_t pk[64];
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) pk[c] = pack2<T>(s[2 * c], s[2 * c + 1]);
-                    tmem_st64(tmem + lane_off + col_p, pk);
+                    if (ok) tmem_st32(tmem + lane_off + col_p + half * 32, pk);
                 }
                 tmem_wait_st();
+                if (!ok) break;
+                const float rsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+                l = fmaf(l, alpha, rsum);
+                m_ref = m_new;
                 tc_fence_before();
                 mbar_arrive(&sh.pv_ready[i]);
             }
             if (!ok) break;
+            if constexpr (Cfg<D>::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
             sh.stat_m[uit & 1][i][t] = m_ref;
             sh.stat_l[uit & 1][i][t] = l;
-            mbar_arrive(&sh.sm2corr[i]);
+            mbar_arrive(&sh.stats_full[i]);
         }
     } else {
         // ================================================================ correction + epilogue
@@ -527,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         constexpr uint32_t kColO[2] = {Cfg<D>::kColO0, Cfg<D>::kColO1};
-        uint32_t c_cnt[2] = {0, 0}, od_cnt[2] = {0, 0}, uit = 0;
+        uint32_t c_cnt[2] = {0, 0}, st_cnt[2] = {0, 0}, od_cnt[2] = {0, 0}, uit = 0;
         bool ok = true;
         auto WS = [&](uint64_t* bar, uint32_t& cnt) {
             if (ok) ok = wait_phase(bar, cnt & 1, abort_flag, p.wait_limit, p.status);
@@ -542,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j >= (i ? U.nkv1 : U.nkv0)) continue;
                     if (j > 0) {
                         if (!WS(&sh.sm2corr[i], c_cnt[i])) break;
-                        const float alpha = sh.alpha[i][t];
+                        const float alpha = sh.alpha[j & 1][i][t];
                         if (!WS(&sh.o_done[i], od_cnt[i])) break;   // PV_i(j-1) complete
                         tc_fence_after();
                         if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -570,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             // epilogue: O = O_acc / l (* sigmoid(G)), lse = (m + log2 l) * ln 2
             for (int i = 0; i < 2; ++i) {
-                if (!WS(&sh.sm2corr[i], c_cnt[i])) break;      // final m, l
+                if (!WS(&sh.stats_full[i], st_cnt[i])) break;  // final m, l
                 if (!WS(&sh.o_done[i], od_cnt[i])) break;      // last PV_i complete
                 tc_fence_after();
                 const float m = sh.stat_m[uit & 1][i][t];
