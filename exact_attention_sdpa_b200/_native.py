@@ -22,7 +22,8 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIM
 ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit", "attn_version")
+EXPORTED = ("attn_fwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+            "attn_debug_inject_stall", "attn_version")
 
 
 class AttnTensor(ctypes.Structure):
@@ -60,6 +61,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_last_device_status.restype = ctypes.c_int
         lib.attn_set_wait_limit.argtypes = [ctypes.c_uint64]
         lib.attn_set_wait_limit.restype = None
+        lib.attn_debug_inject_stall.argtypes = [ctypes.c_int]
+        lib.attn_debug_inject_stall.restype = None
         lib.attn_version.argtypes = []
         lib.attn_version.restype = ctypes.c_char_p
         if path is None:
@@ -168,6 +171,11 @@ def last_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
 
 def set_wait_limit(cycles: int):
     load_library().attn_set_wait_limit(int(cycles))
+
+
+def debug_inject_stall(enable: bool):
+    """Test hook: later launches time out on purpose (see include/attn.h)."""
+    load_library().attn_debug_inject_stall(int(bool(enable)))
 
 
 def version() -> str:

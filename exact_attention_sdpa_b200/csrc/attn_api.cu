@@ -18,6 +18,7 @@ using attn::FwdParams;
 __device__ unsigned int g_status_word;
 
 uint64_t g_wait_limit = 1ull << 32;
+int g_inject_stall = 0;
 
 // ---------------------------------------------------------------------------
 // validation helpers
@@ -271,6 +272,7 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     p.lse = lse;
     p.wait_limit = g_wait_limit;
     p.status = status;
+    p.inject_stall = g_inject_stall;
 
     cudaError_t e;
     if (q->dtype == ATTN_BF16)
@@ -305,6 +307,8 @@ attn_status_t attn_last_device_status(cudaStream_t stream) {
 }
 
 void attn_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles < 1024 ? 1024 : cycles; }
+
+void attn_debug_inject_stall(int enable) { g_inject_stall = enable != 0; }
 
 const char* attn_version(void) { return "0.1.0"; }
 

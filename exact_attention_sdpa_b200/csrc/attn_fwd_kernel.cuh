@@ -79,6 +79,7 @@ struct FwdParams {
     float* lse;                // nullable, [B*H*N]
     unsigned long long wait_limit;
     unsigned int* status;
+    int inject_stall;          // test hook: the MMA warp first waits on a barrier nothing arrives on
 };
 
 template <int D>
@@ -126,6 +127,7 @@ struct __align__(8) FwdShared {
     uint64_t sm2corr[2];     // softmax i -> correction: alpha(j), j >= 1
     uint64_t stats_full[2];  // softmax i -> correction: final m, l of the unit
     uint64_t drain;
+    uint64_t never;          // no arrivals: target of the injected stall
     uint32_t tmem_base;
     int abort_flag;
     float alpha[2][2][kBlockM];    // [iteration parity][tile][row]
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh.v_empty[s], 1);
         }
         mbar_init(&sh.drain, 1);
+        mbar_init(&sh.never, 1);
         sh.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -393,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 return ok;
             };
+            if (p.inject_stall) W(&sh.never, 0);   // gives up after wait_limit cycles: exercises the abort path
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
                 const Unit U = decode_unit<CAUSAL>(u, p);
                 // S0(0), S1(0)

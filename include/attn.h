@@ -110,12 +110,24 @@ attn_status_t attn_last_device_status(cudaStream_t stream);
 
 /*
  * attn_set_wait_limit -- sets the clock-cycle budget of every bounded device
- * wait for later launches on the current device (default 2^32 cycles, about
- * two seconds at 1.9 GHz).  Values below 1024 are raised to 1024.  Tests use a
- * small limit to exercise the timeout path without a fault.  Not thread-safe
- * with concurrent attn_fwd calls.
+ * wait for later launches, process-wide (default 2^32 cycles, about two
+ * seconds at 1.9 GHz).  Values below 1024 are raised to 1024.  A wait whose
+ * phase completes returns as soon as it does; the budget only bounds waits
+ * that would otherwise never end (see attn_debug_inject_stall).  Not
+ * thread-safe with concurrent attn_fwd calls.
  */
 void attn_set_wait_limit(uint64_t cycles);
+
+/*
+ * attn_debug_inject_stall -- test hook for failure detection without a GPU
+ * fault.  While enabled, every later launch on any device makes its MMA warp
+ * first wait on a barrier that nothing arrives on; the bounded wait gives up
+ * after the wait limit (attn_set_wait_limit), records ATTN_ERR_TIMEOUT in the
+ * status word, and every role of the kernel stops, drains its in-flight copies
+ * and MMAs and returns (outputs are then undefined).  Not thread-safe with
+ * concurrent attn_fwd calls.  enable = 0 turns it off.
+ */
+void attn_debug_inject_stall(int enable);
 
 /* The library version as "major.minor.patch" (static string). */
 const char* attn_version(void);
