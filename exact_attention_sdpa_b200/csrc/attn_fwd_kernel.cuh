@@ -123,7 +123,7 @@ struct __align__(8) FwdShared {
     uint64_t s_free[2];      // softmax i -> MMA: S_i(j) read into registers (d <= 64 only)
     uint64_t pv_ready[2];    // softmax i (P written) + correction (O rescaled) -> MMA
     uint64_t o_done[2];      // MMA -> correction: PV_i(j) complete
-    uint64_t o_free[2];      // correction -> MMA: epilogue has read O_i
+    uint64_t o_free[2];      // correction -> MMA and softmax i: epilogue has read O_i and m, l
     uint64_t sm2corr[2];     // softmax i -> correction: alpha(j), j >= 1
     uint64_t stats_full[2];  // softmax i -> correction: final m, l of the unit
     uint64_t drain;
@@ -647,6 +647,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             if constexpr (Cfg<D>::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
+            // The correction must have consumed the previous unit's statistics before this
+            // unit's are published: a unit with a single key tile can otherwise finish before
+            // the correction reaches the previous epilogue, running stats_full two phases ahead.
+            if (uit > 0) {
+                ok = wait_phase(&sh.o_free[i], (uit - 1) & 1, abort_flag, p.wait_limit, p.status);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
             sh.stat_m[uit & 1][i][t] = m_ref;
             sh.stat_l[uit & 1][i][t] = l;
             mbar_arrive(&sh.stats_full[i]);

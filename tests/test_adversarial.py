@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from exact_attention_sdpa_b200 import attn_fwd
+from exact_attention_sdpa_b200 import attn_fwd, last_device_status
 from oracle import sdpa_forward
 from helpers import assert_close_to_oracle, padded
 
@@ -26,6 +26,7 @@ def _check(q, k, v, bias=None, gate=None, causal=False, scale=None, what=""):
     o, lse = attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), None if bias is None else padded(bias, DEV),
                       None if gate is None else gate.to(DEV), causal=causal, scale=scale)
     torch.cuda.synchronize()
+    assert last_device_status() == 0, "a bounded device wait timed out"
     o_ref, l_ref = sdpa_forward(q, k, v, bias=bias, gate=gate, causal=causal, scale=scale)
     assert_close_to_oracle(o, lse, o_ref, l_ref, q.dtype, what)
     return o.cpu(), lse.cpu()
