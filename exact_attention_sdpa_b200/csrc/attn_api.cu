@@ -106,6 +106,29 @@ bool encode_qkv_map(CUtensorMap* map, const attn_tensor_t* t) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bias [H, N, N] or [B, H, N, N] -> 4-D map {keys, rows, H, B}, box {64, 128, 1, 1}, 128-byte swizzle
+bool encode_bias_map(CUtensorMap* map, const attn_tensor_t* b) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (enc == nullptr) return false;
+    const bool has_b = b->ndim == 4;
+    const int64_t H = has_b ? b->shape[1] : b->shape[0];
+    const int64_t N = has_b ? b->shape[2] : b->shape[1];
+    const int64_t si = has_b ? b->stride[2] : b->stride[1];
+    const int64_t sh = has_b ? b->stride[1] : b->stride[0];
+    const int64_t row = N > 1 ? si : 8;
+    const int64_t head = H > 1 ? sh : row * N;
+    const int64_t batch = (has_b && b->shape[0] > 1) ? b->stride[0] : head * H;
+    const cuuint64_t dims[4] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)(has_b ? b->shape[0] : 1)};
+    const cuuint64_t strides[3] = {(cuuint64_t)(row * 2), (cuuint64_t)(head * 2), (cuuint64_t)(batch * 2)};
+    const cuuint32_t box[4] = {64u, 128u, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUtensorMapDataType dt =
+        b->dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return enc(map, dt, 4, b->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
@@ -121,26 +144,28 @@ int sm_count() {
     return counts[dev];
 }
 
+struct Maps {
+    CUtensorMap q, k, v, bias;
+};
+
 template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE>
-cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-                     cudaStream_t stream) {
+cudaError_t launch_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
     auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE>;
-    constexpr int smem = attn::Cfg<D>::kDynBytes;
+    constexpr int smem = attn::BiasCfg<D, BIAS>::kDynBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
     // persistent: one CTA per SM (tensor memory and registers allow no more)
     const int grid = p.num_units < sms ? p.num_units : sms;
-    kern<<<grid, attn::kThreads, smem, stream>>>(mq, mk, mv, p);
+    kern<<<grid, attn::kThreads, smem, stream>>>(m.q, m.k, m.v, m.bias, p);
     return cudaGetLastError();
 }
 
 template <typename T, int D>
-cudaError_t launch_d(bool causal, bool bias, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
-                     const CUtensorMap& mv, const FwdParams& p, cudaStream_t s) {
+cudaError_t launch_d(bool causal, bool bias, bool gate, const Maps& m, const FwdParams& p, cudaStream_t s) {
 #define ATTN_CASE(C, B_, G_) \
-    if (causal == C && bias == B_ && gate == G_) return launch_t<T, D, C, B_, G_>(mq, mk, mv, p, s);
+    if (causal == C && bias == B_ && gate == G_) return launch_t<T, D, C, B_, G_>(m, p, s);
     ATTN_CASE(false, false, false)
     ATTN_CASE(false, false, true)
     ATTN_CASE(false, true, false)
@@ -154,12 +179,12 @@ cudaError_t launch_d(bool causal, bool bias, bool gate, const CUtensorMap& mq, c
 }
 
 template <typename T>
-cudaError_t launch_dtype(int d, bool causal, bool bias, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const FwdParams& p, cudaStream_t s) {
+cudaError_t launch_dtype(int d, bool causal, bool bias, bool gate, const Maps& m, const FwdParams& p,
+                         cudaStream_t s) {
     switch (d) {
-        case 32: return launch_d<T, 32>(causal, bias, gate, mq, mk, mv, p, s);
-        case 64: return launch_d<T, 64>(causal, bias, gate, mq, mk, mv, p, s);
-        case 128: return launch_d<T, 128>(causal, bias, gate, mq, mk, mv, p, s);
+        case 32: return launch_d<T, 32>(causal, bias, gate, m, p, s);
+        case 64: return launch_d<T, 64>(causal, bias, gate, m, p, s);
+        case 128: return launch_d<T, 128>(causal, bias, gate, m, p, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -231,8 +256,12 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
 
     // ---- launch
-    CUtensorMap mq, mk, mv;
-    if (!encode_qkv_map(&mq, q) || !encode_qkv_map(&mk, k) || !encode_qkv_map(&mv, v)) return ATTN_ERR_CUDA;
+    Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!encode_qkv_map(&maps.q, q) || !encode_qkv_map(&maps.k, k) || !encode_qkv_map(&maps.v, v))
+        return ATTN_ERR_CUDA;
+    // d <= 64 stages bias tiles through shared memory by TMA; d = 128 reads bias rows directly
+    if (bias != nullptr && d <= 64 && !encode_bias_map(&maps.bias, bias)) return ATTN_ERR_CUDA;
     unsigned int* status = status_word_ptr();
     if (status == nullptr) return ATTN_ERR_CUDA;
 
@@ -276,11 +305,11 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
 
     cudaError_t e;
     if (q->dtype == ATTN_BF16)
-        e = launch_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, mq, mk,
-                                        mv, p, stream);
+        e = launch_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, maps, p,
+                                        stream);
     else
-        e = launch_dtype<__half>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, mq, mk, mv,
-                                 p, stream);
+        e = launch_dtype<__half>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, maps, p,
+                                 stream);
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

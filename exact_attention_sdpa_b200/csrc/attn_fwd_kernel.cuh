@@ -113,6 +113,29 @@ struct Cfg {
     static constexpr int kBytes = kOffV + kStages * kTileBytes;
     static constexpr int kDynBytes = kBytes + 1024;
     static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
+    // per-thread registers after setmaxnreg: 256 softmax + 128 correction + 128 other
+    // threads must fit the 65536 the CTA was launched with (512 threads x 128)
+    static constexpr int kRegsSoftmax = 176;
+    static constexpr int kRegsCorrection = (D == 128) ? 80 : 88;
+    static constexpr int kRegsOther = (D == 128) ? 80 : 72;
+    static_assert(256 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= 65536, "register budget");
+};
+
+// Additive bias staged through shared memory by TMA (d <= 64; at d = 128 the K/V rings
+// leave no room and each softmax thread reads its bias row from global memory).  A bias
+// tile is 128 query rows x 128 keys of 16-bit values, stored as two 128 x 64 boxes with
+// the 128-byte swizzle, so that thread t reading 16-byte chunk k of its row touches
+// chunk position k ^ (t & 7): conflict-free.
+template <int D, bool HAS_BIAS>
+struct BiasCfg {
+    static constexpr bool kTma = HAS_BIAS && D <= 64;
+    static constexpr int kStages = (D == 32) ? 2 : 1;
+    static constexpr int kBoxBytes = kBlockM * 64 * 2;            // 16 KB
+    static constexpr int kTileBytes = 2 * kBoxBytes;               // 32 KB
+    static constexpr int kOff = Cfg<D>::kBytes;
+    static constexpr int kBytes = kTma ? 2 * kStages * kTileBytes : 0;
+    static constexpr int kDynBytes = Cfg<D>::kBytes + kBytes + 1024;
+    static_assert(kDynBytes <= 214 * 1024, "shared memory budget (dynamic + static)");
 };
 
 template <int ST>
@@ -128,6 +151,7 @@ struct __align__(8) FwdShared {
     uint64_t stats_full[2];  // softmax i -> correction: final m, l of the unit
     uint64_t drain;
     uint64_t never;          // no arrivals: target of the injected stall
+    uint64_t bias_full[2][2], bias_empty[2][2];   // [tile][stage], staged bias tiles
     uint32_t tmem_base;
     int abort_flag;
     float alpha[2][2][kBlockM];    // [iteration parity][tile][row]
@@ -231,7 +255,8 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
 template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
+                    const FwdParams p) {
     using namespace sm100;
     using C = Cfg<D>;
     constexpr int ST = C::kStages;
@@ -243,6 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
+    using BC = BiasCfg<D, HAS_BIAS>;
+    uint8_t* sBias = smem + BC::kOff;      // [tile][stage][2 boxes]
 
     const int warp = warp_id();
     const int lane = lane_id();
@@ -268,6 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sh.drain, 1);
         mbar_init(&sh.never, 1);
+        for (int i = 0; i < 2; ++i)
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&sh.bias_full[i][b], 1);
+                mbar_init(&sh.bias_empty[i][b], kBlockM);
+            }
         sh.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -283,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* abort_flag = &sh.abort_flag;
 
     if (wg == 3) {
-        regs_dec<80>();
+        regs_dec<Cfg<D>::kRegsOther>();
         if (warp == 13) {
             // ============================================================ TMA producer
             // The whole warp runs this loop (uniform control flow); one elected lane issues.
@@ -313,6 +345,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 ++qc[i];
             };
+            uint32_t bc[2] = {0, 0};            // bias tiles loaded per query tile
+            auto load_bias = [&](int i, int j, const Unit& U) {
+                const uint32_t st = bc[i] % BC::kStages;
+                if (bc[i] >= BC::kStages &&
+                    !WU(&sh.bias_empty[i][st], ((bc[i] / BC::kStages) - 1) & 1))
+                    return;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&sh.bias_full[i][st], BC::kTileBytes);
+                    uint8_t* dst = sBias + (i * BC::kStages + st) * BC::kTileBytes;
+                    const int bb = p.bias_sb != 0 ? U.b : 0;
+                    for (int half = 0; half < 2; ++half)
+                        tma_load_4d(dst + half * BC::kBoxBytes, &tm_bias, &sh.bias_full[i][st],
+                                    j * kBlockN + half * 64, U.q0 + i * kBlockM, U.h, bb, pol_kv);
+                }
+                __syncwarp();
+                ++bc[i];
+            };
             auto load_kv = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, const CUtensorMap* map, uint32_t& cnt,
                                int j, const Unit& U) {
                 const uint32_t st = cnt % ST;
@@ -332,9 +381,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, 0, U);
                 if (ok) load_q(1, U);
                 if (ok) load_kv(sh.v_full, sh.v_empty, sV, &tm_v, vc, 0, U);
+                if constexpr (BC::kTma) {
+                    if (ok) load_bias(0, 0, U);
+                    if (ok) load_bias(1, 0, U);
+                }
                 for (int j = 1; ok && j < U.nkv1; ++j) {
                     load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, j, U);
                     if (ok) load_kv(sh.v_full, sh.v_empty, sV, &tm_v, vc, j, U);
+                    if constexpr (BC::kTma) {
+                        if (ok && j < U.nkv0) load_bias(0, j, U);
+                        if (ok) load_bias(1, j, U);
+                    }
                 }
             }
             // drain: every load issued into shared memory lands before the CTA exits
@@ -343,6 +400,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (uint32_t s = 0; s < ST; ++s) {
                 if (kc > s) drain_phase(&sh.k_full[s], ((kc - 1 - s) / ST) & 1, p.status);
                 if (vc > s) drain_phase(&sh.v_full[s], ((vc - 1 - s) / ST) & 1, p.status);
+            }
+            if constexpr (BC::kTma) {
+                for (int i = 0; i < 2; ++i)
+                    for (uint32_t s = 0; s < (uint32_t)BC::kStages; ++s)
+                        if (bc[i] > s)
+                            drain_phase(&sh.bias_full[i][s], ((bc[i] - 1 - s) / BC::kStages) & 1, p.status);
             }
         } else if (warp == 12) {
             // ============================================================ MMA issuer
@@ -397,25 +460,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return ok;
             };
             if (p.inject_stall) W(&sh.never, 0);   // gives up after wait_limit cycles: exercises the abort path
+            // S_i(0) of a unit: Q_i of that unit and its first key tile (ring position kpos)
+            auto issue_first_s = [&](int i, int nkv_i, uint32_t kpos, uint32_t qpar) -> bool {
+                if (!W(&sh.q_full[i], qpar) || !W(&sh.k_full[kpos % ST], (kpos / ST) & 1)) return false;
+                tc_fence_after();
+                issue_s(i, kpos % ST);
+                commit(&sh.s_full[i]);
+                if (i == 1) commit(&sh.k_empty[kpos % ST]);
+                if (nkv_i == 1) commit(&sh.q_empty[i]);
+                return true;
+            };
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
                 const Unit U = decode_unit<CAUSAL>(u, p);
-                // S0(0), S1(0)
-                if (!W(&sh.q_full[0], uit & 1) || !W(&sh.k_full[kc % ST], (kc / ST) & 1)) break;
-                tc_fence_after();
-                issue_s(0, kc % ST);
-                commit(&sh.s_full[0]);
-                if (U.nkv0 == 1) commit(&sh.q_empty[0]);
-                if (!W(&sh.q_full[1], uit & 1)) break;
-                tc_fence_after();
-                issue_s(1, kc % ST);
-                commit(&sh.s_full[1]);
-                commit(&sh.k_empty[kc % ST]);
-                if (U.nkv1 == 1) commit(&sh.q_empty[1]);
+                const int un = u + static_cast<int>(gridDim.x);
+                const bool has_next = un < p.num_units;
+                // S0(0), S1(0): d <= 64 issues them for later units during the previous unit
+                if (!C::kSeparateP || uit == 0) {
+                    if (!issue_first_s(0, U.nkv0, kc, uit & 1) || !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
+                }
                 for (int j = 0; j < U.nkv1; ++j) {
                     const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
                     const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
                     if constexpr (C::kSeparateP) {
                         // S0(j+1), S1(j+1) as soon as the softmax has read S(j); then PV0(j), PV1(j)
+                        // (at the last iteration of a tile: S_i(0) of the next unit instead)
                         if (j + 1 < U.nkv0) {
                             if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
                             ++sf_cnt[0];
@@ -424,6 +492,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             issue_s(0, kst);
                             commit(&sh.s_full[0]);
                             if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
+                        } else if (j + 1 == U.nkv0 && has_next) {
+                            if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
+                            ++sf_cnt[0];
+                            if (!issue_first_s(0, decode_unit<CAUSAL>(un, p).nkv0, kc + U.nkv1, (uit + 1) & 1)) break;
                         }
                         if (j + 1 < U.nkv1) {
                             if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
@@ -434,6 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             commit(&sh.s_full[1]);
                             commit(&sh.k_empty[kst]);
                             if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
+                        } else if (has_next) {
+                            if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
+                            ++sf_cnt[1];
+                            if (!issue_first_s(1, decode_unit<CAUSAL>(un, p).nkv1, kc + U.nkv1, (uit + 1) & 1)) break;
                         }
                         if (j < U.nkv0) {
                             if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
@@ -498,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (wg < 2) {
         // ================================================================ softmax of tile i = wg
-        regs_inc<176>();
+        regs_inc<Cfg<D>::kRegsSoftmax>();
         const int i = wg;
         const int t = threadIdx.x & 127;          // row within the tile
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -506,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t col_p = i ? Cfg<D>::kColP1 : Cfg<D>::kColP0;
         const float scale_log2 = p.scale_log2;
         const bool fast = !HAS_BIAS && scale_log2 > 0.f;   // max over raw scores, fused scale
-        uint32_t s_cnt = 0, od_cnt = 0, uit = 0;
+        uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
             const Unit U = decode_unit<CAUSAL>(u, p);
@@ -536,7 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(r[c]);
                 }
                 if constexpr (Cfg<D>::kSeparateP) {
-                    if (j + 1 < nkv) {      // S_i may now be overwritten by S_i(j+1)
+                    // S_i may now be overwritten by S_i(j+1), or by S_i(0) of the next unit
+                    if (j + 1 < nkv || u + static_cast<int>(gridDim.x) < p.num_units) {
                         tc_fence_before();
                         mbar_arrive(&sh.s_free[i]);
                     }
@@ -552,10 +629,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     m_tile = row_max(s) * scale_log2;
                 } else {
+                    const uint8_t* brow = nullptr;
+                    uint32_t bst = 0;
+                    if constexpr (BC::kTma) {
+                        bst = bcnt % BC::kStages;
+                        ok = wait_phase(&sh.bias_full[i][bst], (bcnt / BC::kStages) & 1, abort_flag, p.wait_limit,
+                                        p.status);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        brow = sBias + (i * BC::kStages + bst) * BC::kTileBytes + t * 128;
+                    }
 #pragma unroll
                     for (int c = 0; c < kBlockN; c += 8) {
                         float bv[8];
-                        if constexpr (HAS_BIAS) {
+                        if constexpr (BC::kTma) {
+                            // chunk (c % 64) / 8 of box c / 64, 128-byte swizzle
+                            const uint4 raw = *reinterpret_cast<const uint4*>(
+                                brow + (c / 64) * BC::kBoxBytes + ((((c % 64) / 8) ^ (t & 7)) << 4));
+                            const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) bv[q] = to_f32<T>(e[q]);
+                        } else if constexpr (HAS_BIAS) {
                             if (row < p.N && kv0 + c + 8 <= p.N) {
                                 const uint4 raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
                                 const T* e = reinterpret_cast<const T*>(&raw);
@@ -573,6 +667,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if constexpr (HAS_BIAS) x = fmaf(bv[q], kLog2e, x);
                             s[c + q] = x;
                         }
+                    }
+                    if constexpr (BC::kTma) {          // the staged bias tile may be refilled
+                        mbar_arrive(&sh.bias_empty[i][bst]);
+                        ++bcnt;
                     }
                     if (need_mask) {
                         const int lim = CAUSAL ? min(p.N - kv0, row - kv0 + 1) : (p.N - kv0);
@@ -624,15 +722,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // P_i(j) overwrites P_i(j-1): PV_i(j-1) must have completed.  Its
                         // completion also means the correction consumed alpha(j-1), so alpha(j)
                         // is published only now (its barrier never runs two phases ahead).
-                        if (half == 0 && j > 0) {
+                        // (iteration 0 of a later unit: the previous unit's last PV_i, which the
+                        // MMA warp issues after this unit's S_i(0))
+                        if (half == 0 && (j > 0 || uit > 0)) {
                             ok = wait_phase(&sh.o_done[i], od_cnt & 1, abort_flag, p.wait_limit, p.status);
                             ++od_cnt;
                             ok = __all_sync(0xffffffffu, ok);
-                            if (ok) {
-                                tc_fence_after();
-                                sh.alpha[j & 1][i][t] = alpha;
-                                mbar_arrive(&sh.sm2corr[i]);
-                            }
+                            if (ok) tc_fence_after();
+                        }
+                        if (half == 0 && j > 0 && ok) {
+                            sh.alpha[j & 1][i][t] = alpha;
+                            mbar_arrive(&sh.sm2corr[i]);
                         }
                     }
                     if (ok) tmem_st32(tmem + lane_off + col_p + half * 32, pk);
@@ -646,7 +746,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&sh.pv_ready[i]);
             }
             if (!ok) break;
-            if constexpr (Cfg<D>::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
             // The correction must have consumed the previous unit's statistics before this
             // unit's are published: a unit with a single key tile can otherwise finish before
             // the correction reaches the previous epilogue, running stats_full two phases ahead.
@@ -661,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================================ correction + epilogue
-        regs_dec<80>();
+        regs_dec<Cfg<D>::kRegsCorrection>();
         const int t = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         constexpr uint32_t kColO[2] = {Cfg<D>::kColO0, Cfg<D>::kColO1};
@@ -701,59 +800,80 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tmem_wait_st();
                         }
                         tc_fence_before();
+                        mbar_arrive(&sh.pv_ready[i]);
+                    } else if (uit == 0) {
+                        mbar_arrive(&sh.pv_ready[i]);   // later units: arrived by the previous epilogue
                     }
-                    mbar_arrive(&sh.pv_ready[i]);
                 }
             }
             if (!ok) break;
-            // epilogue: O = O_acc / l (* sigmoid(G)), lse = (m + log2 l) * ln 2
+            // epilogue: O = O_acc / l (* sigmoid(G)), lse = (m + log2 l) * ln 2.
+            // O_i is released as soon as its last chunk is in registers, together with the next
+            // unit's first pv_ready arrival (iteration 0 needs no rescale), so the next unit's
+            // PV_i(0) does not wait for the gate arithmetic and global stores.
+            const bool has_next = u + static_cast<int>(gridDim.x) < p.num_units;
             for (int i = 0; i < 2; ++i) {
-                if (!WS(&sh.stats_full[i], st_cnt[i])) break;  // final m, l
-                if (!WS(&sh.o_done[i], od_cnt[i])) break;      // last PV_i complete
-                tc_fence_after();
-                const float m = sh.stat_m[uit & 1][i][t];
-                const float l = sh.stat_l[uit & 1][i][t];
                 const int row = U.q0 + i * kBlockM + t;
                 const bool row_ok = row < p.N;
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
                 T* orow = reinterpret_cast<T*>(p.out) + U.b * p.out_sb + U.h * p.out_sh +
                           static_cast<int64_t>(row_ok ? row : 0) * p.out_si;
                 const T* grow = nullptr;
                 if constexpr (HAS_GATE)
                     grow = reinterpret_cast<const T*>(p.gate) + U.b * p.gate_sb + U.h * p.gate_sh +
                            static_cast<int64_t>(row_ok ? row : 0) * p.gate_si;
+                constexpr int kPre = (HAS_GATE && D == 32) ? D / 8 : 1;   // gate row prefetched (d = 32)
+                uint4 graw[kPre];
+                if constexpr (HAS_GATE && D == 32) {
+                    if (row_ok) {
+#pragma unroll
+                        for (int v8 = 0; v8 < D / 8; ++v8) graw[v8] = __ldg(reinterpret_cast<const uint4*>(grow + v8 * 8));
+                    }
+                }
+                if (!WS(&sh.stats_full[i], st_cnt[i])) break;  // final m, l
+                if (!WS(&sh.o_done[i], od_cnt[i])) break;      // last PV_i complete
+                tc_fence_after();
+                const float m = sh.stat_m[uit & 1][i][t];
+                const float l = sh.stat_l[uit & 1][i][t];
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                // one 32-column chunk of O: normalise, gate, round, store
+                auto finish_chunk = [&](const uint32_t (&r)[32], int c) {
+                    if (!row_ok) return;
+#pragma unroll
+                    for (int v8 = 0; v8 < 4; ++v8) {
+                        float o[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) o[q] = __uint_as_float(r[v8 * 8 + q]) * inv_l;
+                        if constexpr (HAS_GATE) {
+                            uint4 raw;
+                            if constexpr (D == 32) raw = graw[v8];
+                            else raw = __ldg(reinterpret_cast<const uint4*>(grow + c * 32 + v8 * 8));
+                            const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) o[q] *= 1.f / (1.f + ex2_approx(-to_f32<T>(e[q]) * kLog2e));
+                        }
+                        uint4 w;
+                        w.x = pack2<T>(o[0], o[1]);
+                        w.y = pack2<T>(o[2], o[3]);
+                        w.z = pack2<T>(o[4], o[5]);
+                        w.w = pack2<T>(o[6], o[7]);
+                        *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = w;
+                    }
+                };
                 uint32_t r[32];
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     tmem_ld32(tmem + lane_off + kColO[i] + c * 32, r);
                     tmem_wait_ld(r);
-                    if (row_ok) {
-#pragma unroll
-                        for (int v8 = 0; v8 < 4; ++v8) {
-                            float o[8];
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) o[q] = __uint_as_float(r[v8 * 8 + q]) * inv_l;
-                            if constexpr (HAS_GATE) {
-                                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(grow + c * 32 + v8 * 8));
-                                const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-                                for (int q = 0; q < 8; ++q)
-                                    o[q] *= 1.f / (1.f + ex2_approx(-to_f32<T>(e[q]) * kLog2e));
-                            }
-                            uint4 w;
-                            w.x = pack2<T>(o[0], o[1]);
-                            w.y = pack2<T>(o[2], o[3]);
-                            w.z = pack2<T>(o[4], o[5]);
-                            w.w = pack2<T>(o[6], o[7]);
-                            *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = w;
-                        }
+                    if (c == D / 32 - 1) {        // O_i fully read: release it
+                        tc_fence_before();
+                        mbar_arrive(&sh.o_free[i]);
+                        if (has_next) mbar_arrive(&sh.pv_ready[i]);
                     }
+                    finish_chunk(r, c);
                 }
                 if (p.lse != nullptr && row_ok)
                     p.lse[static_cast<int64_t>(U.bh) * p.N + row] =
                         (l > 0.f) ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
-                tc_fence_before();
-                mbar_arrive(&sh.o_free[i]);
             }
         }
     }
