@@ -472,18 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
                 const Unit U = decode_unit<CAUSAL>(u, p);
-                const int un = u + static_cast<int>(gridDim.x);
-                const bool has_next = un < p.num_units;
-                // S0(0), S1(0): d <= 64 issues them for later units during the previous unit
-                if (!C::kSeparateP || uit == 0) {
-                    if (!issue_first_s(0, U.nkv0, kc, uit & 1) || !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
-                }
+                // S0(0), S1(0)
+                if (!issue_first_s(0, U.nkv0, kc, uit & 1) || !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
                 for (int j = 0; j < U.nkv1; ++j) {
                     const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
                     const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
                     if constexpr (C::kSeparateP) {
                         // S0(j+1), S1(j+1) as soon as the softmax has read S(j); then PV0(j), PV1(j)
-                        // (at the last iteration of a tile: S_i(0) of the next unit instead)
                         if (j + 1 < U.nkv0) {
                             if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
                             ++sf_cnt[0];
@@ -492,10 +487,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             issue_s(0, kst);
                             commit(&sh.s_full[0]);
                             if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
-                        } else if (j + 1 == U.nkv0 && has_next) {
-                            if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
-                            ++sf_cnt[0];
-                            if (!issue_first_s(0, decode_unit<CAUSAL>(un, p).nkv0, kc + U.nkv1, (uit + 1) & 1)) break;
                         }
                         if (j + 1 < U.nkv1) {
                             if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
@@ -506,10 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             commit(&sh.s_full[1]);
                             commit(&sh.k_empty[kst]);
                             if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
-                        } else if (has_next) {
-                            if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
-                            ++sf_cnt[1];
-                            if (!issue_first_s(1, decode_unit<CAUSAL>(un, p).nkv1, kc + U.nkv1, (uit + 1) & 1)) break;
                         }
                         if (j < U.nkv0) {
                             if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
@@ -612,8 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(r[c]);
                 }
                 if constexpr (Cfg<D>::kSeparateP) {
-                    // S_i may now be overwritten by S_i(j+1), or by S_i(0) of the next unit
-                    if (j + 1 < nkv || u + static_cast<int>(gridDim.x) < p.num_units) {
+                    // S_i may now be overwritten by S_i(j+1) (S_i(0) of the next unit is issued
+                    // only after this unit's last PV_i, which needs this softmax to finish)
+                    if (j + 1 < nkv) {
                         tc_fence_before();
                         mbar_arrive(&sh.s_free[i]);
                     }
@@ -722,9 +710,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // P_i(j) overwrites P_i(j-1): PV_i(j-1) must have completed.  Its
                         // completion also means the correction consumed alpha(j-1), so alpha(j)
                         // is published only now (its barrier never runs two phases ahead).
-                        // (iteration 0 of a later unit: the previous unit's last PV_i, which the
-                        // MMA warp issues after this unit's S_i(0))
-                        if (half == 0 && (j > 0 || uit > 0)) {
+                        // (iteration 0 needs no wait: S_i(0) was issued after the previous unit's
+                        // last PV_i, and its commit covers that PV)
+                        if (half == 0 && j > 0) {
                             ok = wait_phase(&sh.o_done[i], od_cnt & 1, abort_flag, p.wait_limit, p.status);
                             ++od_cnt;
                             ok = __all_sync(0xffffffffu, ok);
@@ -749,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The correction must have consumed the previous unit's statistics before this
             // unit's are published: a unit with a single key tile can otherwise finish before
             // the correction reaches the previous epilogue, running stats_full two phases ahead.
+            if constexpr (Cfg<D>::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
             if (uit > 0) {
                 ok = wait_phase(&sh.o_free[i], (uit - 1) & 1, abort_flag, p.wait_limit, p.status);
                 ok = __all_sync(0xffffffffu, ok);
