@@ -132,6 +132,18 @@ bool encode_bias_map(CUtensorMap* map, const attn_tensor_t* b) {
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
+int l2_bytes() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    static int sizes[64] = {0};
+    if (sizes[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev) != cudaSuccess) return 0;
+        sizes[dev] = n;
+    }
+    return sizes[dev];
+}
+
 int sm_count() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
@@ -276,6 +288,15 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
     p.num_units = static_cast<int>(units);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    // unit order: when the K/V of all heads exceed the L2, schedule a few heads at a
+    // time (enough query pairs to occupy every SM), else all heads together
+    {
+        const double kv_bytes = 2.0 * static_cast<double>(B * H) * static_cast<double>(N) * d * 2.0;
+        const int sms = sm_count();
+        int g = static_cast<int>(B * H);
+        if (sms > 0 && kv_bytes > static_cast<double>(l2_bytes())) g = (sms + p.num_q_pairs - 1) / p.num_q_pairs;
+        p.head_group = g < 1 ? 1 : (g > B * H ? static_cast<int>(B * H) : g);
+    }
     if (bias != nullptr) {
         p.bias = bias->data;
         if (bias->ndim == 3) {

@@ -69,6 +69,7 @@ struct FwdParams {
     int num_q_pairs;           // ceil(N / 256)
     int num_units;             // num_q_pairs * B * H
     int n_kv_tiles;            // ceil(N / 128)
+    int head_group;            // heads per scheduling group (see decode_unit)
     float scale_log2;          // scale * log2(e)
     const void* bias;          // nullable
     int64_t bias_sb, bias_sh, bias_si;   // element strides (bias_sb = 0 when shared over B)
@@ -238,8 +239,17 @@ template <bool CAUSAL>
 __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
     Unit U;
     const int BH = p.B * p.H;
-    U.qp = p.num_q_pairs - 1 - u / BH;     // heaviest query pairs first
-    U.bh = u % BH;
+    // Units are taken in groups of `head_group` heads; inside a group the heaviest query
+    // pairs come first (causal load balance).  With head_group = B*H (the default) this is
+    // one group: heaviest pairs of all heads first.  For long sequences whose K/V do not
+    // fit in L2 the host picks a small group, so that the CTAs running at the same time
+    // share the K/V of a few heads in L2 instead of streaming all of them from DRAM.
+    const int G = p.head_group;
+    const int per = G * p.num_q_pairs;
+    const int g = u / per, r = u % per;
+    const int gsize = min(G, BH - g * G);       // the last group may be partial
+    U.qp = p.num_q_pairs - 1 - r / gsize;
+    U.bh = g * G + r % gsize;
     U.b = U.bh / p.H;
     U.h = U.bh % p.H;
     U.q0 = U.qp * kRowsPerUnit;

@@ -131,3 +131,16 @@ def test_deterministic(name):
 def test_batch_heads_many():
     w = Workload("bh", B=5, H=7, N=160, d=64, dtype="fp16", causal=True, seed=21)
     _full_check(w)
+
+
+def test_head_grouped_order_with_partial_group():
+    """Long sequences whose K/V exceed the L2 are scheduled a few heads at a time;
+    9 heads at N=32768 (302 MB of K/V) form groups of 2 and a partial group of 1."""
+    w = Workload("grouped", B=1, H=9, N=32768, d=128, dtype="bf16", causal=True, seed=31, amp=0.5)
+    inp = make_inputs(w)
+    o, lse = _run(inp, w)
+    picks = _sampled_rows(w, n_bh=5)
+    picks += [(0, h, i) for h in range(9) for i in (0, 255, 256, 16383, 32767)]
+    o_ref, l_ref = sdpa_rows(inp["q"], inp["k"], inp["v"], picks, causal=True, scale=w.scale)
+    idx = tuple(np.array(x) for x in zip(*picks))
+    assert_close_to_oracle(o.cpu()[idx], lse.cpu()[idx], o_ref, l_ref, torch.bfloat16, "grouped")
