@@ -287,6 +287,7 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     const int64_t units = static_cast<int64_t>(p.num_q_pairs) * B * H;
     if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
     p.num_units = static_cast<int>(units);
+    p.scale = scale;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     // unit order: when the K/V of all heads exceed the L2, schedule a few heads at a
     // time (enough query pairs to occupy every SM), else all heads together

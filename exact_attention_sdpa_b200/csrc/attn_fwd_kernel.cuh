@@ -70,6 +70,7 @@ struct FwdParams {
     int num_units;             // num_q_pairs * B * H
     int n_kv_tiles;            // ceil(N / 128)
     int head_group;            // heads per scheduling group (see decode_unit)
+    float scale;               // multiplies Q K^T
     float scale_log2;          // scale * log2(e)
     const void* bias;          // nullable
     int64_t bias_sb, bias_sh, bias_si;   // element strides (bias_sb = 0 when shared over B)
@@ -637,33 +638,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         brow = sBias + (i * BC::kStages + bst) * BC::kTileBytes + t * 128;
                     }
+                    // y = scale * s + bias in natural units, one packed FMA per pair; the
+                    // conversion to log2 units rides on the exponent's FMA below
+                    const float sc = p.scale;
 #pragma unroll
                     for (int c = 0; c < kBlockN; c += 8) {
-                        float bv[8];
-                        if constexpr (BC::kTma) {
-                            // chunk (c % 64) / 8 of box c / 64, 128-byte swizzle
-                            const uint4 raw = *reinterpret_cast<const uint4*>(
-                                brow + (c / 64) * BC::kBoxBytes + ((((c % 64) / 8) ^ (t & 7)) << 4));
-                            const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) bv[q] = to_f32<T>(e[q]);
-                        } else if constexpr (HAS_BIAS) {
-                            if (row < p.N && kv0 + c + 8 <= p.N) {
-                                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
-                                const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) bv[q] = to_f32<T>(e[q]);
+                        if constexpr (HAS_BIAS) {
+                            uint4 raw;
+                            if constexpr (BC::kTma) {
+                                // chunk (c % 64) / 8 of box c / 64, 128-byte swizzle
+                                raw = *reinterpret_cast<const uint4*>(
+                                    brow + (c / 64) * BC::kBoxBytes + ((((c % 64) / 8) ^ (t & 7)) << 4));
+                            } else if (row < p.N && kv0 + c + 8 <= p.N) {
+                                raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
                             } else {
+                                T e[8];
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
-                                    bv[q] = (row < p.N && kv0 + c + q < p.N) ? to_f32<T>(bias_row[kv0 + c + q]) : 0.f;
+                                    e[q] = (row < p.N && kv0 + c + q < p.N) ? bias_row[kv0 + c + q] : T(0.f);
+                                raw = *reinterpret_cast<const uint4*>(e);
                             }
-                        }
+                            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float x = s[c + q] * scale_log2;
-                            if constexpr (HAS_BIAS) x = fmaf(bv[q], kLog2e, x);
-                            s[c + q] = x;
+                            for (int q = 0; q < 4; ++q) {
+                                float b0, b1;
+                                unpack2<T>(w[q], b0, b1);
+                                ffma2(s[c + 2 * q], s[c + 2 * q + 1], s[c + 2 * q], s[c + 2 * q + 1], sc, sc, b0, b1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 8; q += 2)
+                                fmul2(s[c + q], s[c + q + 1], s[c + q], s[c + q + 1], sc, sc);
                         }
                     }
                     if constexpr (BC::kTma) {          // the staged bias tile may be refilled
@@ -675,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
                     }
-                    m_tile = row_max(s);
+                    m_tile = row_max(s) * kLog2e;
                 }
                 // reference maximum: move it only when the row maximum grew by more than the threshold
                 float m_new = m_ref, alpha = 1.f;
@@ -692,10 +697,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&sh.sm2corr[i]);
                 }
                 const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                // p = 2^(x - m): x = s * scale_log2 on the fast path (s raw), x = s otherwise.
+                // p = 2^(x - m): x = s * scale_log2 on the fast path (s raw), x = y * log2(e) otherwise.
                 // One pair in three goes through the FMA-pipe exponential so that the
                 // MUFU unit (16 lanes per clock per SM) is not the only exp resource.
-                const float xa = fast ? scale_log2 : 1.f;
+                const float xa = fast ? scale_log2 : kLog2e;
                 const float xb = -m_use;
                 float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
