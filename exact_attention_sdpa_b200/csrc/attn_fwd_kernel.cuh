@@ -118,8 +118,8 @@ struct Cfg {
     // per-thread registers after setmaxnreg: 256 softmax + 128 correction + 128 other
     // threads must fit the 65536 the CTA was launched with (512 threads x 128)
     static constexpr int kRegsSoftmax = 176;
-    static constexpr int kRegsCorrection = (D == 128) ? 80 : 88;
-    static constexpr int kRegsOther = (D == 128) ? 80 : 72;
+    static constexpr int kRegsCorrection = 80;
+    static constexpr int kRegsOther = 80;
     static_assert(256 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= 65536, "register budget");
 };
 
@@ -235,6 +235,15 @@ __device__ __forceinline__ void ex2_emu2(float& y0, float& y1, float x0, float x
 struct Unit {
     int b, h, bh, qp, q0, nkv0, nkv1;
 };
+
+// The k-th unit a CTA processes.  Wave k (the k-th unit of every CTA) takes units
+// [k G, (k+1) G) of the heaviest-first order, G = gridDim.x, forwards for even k and
+// backwards for odd k: the CTA that drew the heaviest unit of one wave draws the
+// lightest of the next, which evens out the per-CTA totals of causal workloads.
+__device__ __forceinline__ int unit_at(int k) {
+    const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    return k * G + ((k & 1) ? (G - 1 - b) : b);
+}
 
 template <bool CAUSAL>
 __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
@@ -386,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 ++cnt;
             };
-            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+            for (int k = 0, u = unit_at(0); ok && u < p.num_units; u = unit_at(++k)) {
                 const Unit U = decode_unit<CAUSAL>(u, p);
                 load_q(0, U);
                 if (ok) load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, 0, U);
@@ -481,10 +490,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (nkv_i == 1) commit(&sh.q_empty[i]);
                 return true;
             };
-            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
+            // d <= 64 issues S_i(0) of the next unit right after this unit's last PV_i rather than
+            // after both tiles' last PVs, so tile 0's softmax restarts one PV group earlier.
+            // Issued after that PV, S_i(0) needs no further ordering: its commit covers the PV.
+            bool early[2] = {false, false};
+            for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
                 const Unit U = decode_unit<CAUSAL>(u, p);
-                // S0(0), S1(0)
-                if (!issue_first_s(0, U.nkv0, kc, uit & 1) || !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
+                const int u_next = unit_at(uit + 1);
+                int nkv_next[2] = {0, 0};      // 0: no next unit
+                if (C::kSeparateP && u_next < p.num_units) {
+                    const Unit Un = decode_unit<CAUSAL>(u_next, p);
+                    nkv_next[0] = Un.nkv0;
+                    nkv_next[1] = Un.nkv1;
+                }
+                // S0(0), S1(0), unless issued at the end of the previous unit
+                if (!early[0] && !issue_first_s(0, U.nkv0, kc, uit & 1)) break;
+                if (!early[1] && !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
+                early[0] = early[1] = false;
                 for (int j = 0; j < U.nkv1; ++j) {
                     const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
                     const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
@@ -517,6 +539,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                             issue_pv(0, vst, j > 0);
                             commit(&sh.o_done[0]);
+                            if (j + 1 == U.nkv0 && nkv_next[0] > 0) {
+                                if (!issue_first_s(0, nkv_next[0], kc + U.nkv1, (uit + 1) & 1))
+                                    break;
+                                early[0] = true;
+                            }
                         }
                         if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
                         ++pv_cnt[1];
@@ -526,6 +553,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         issue_pv(1, vst, j > 0);
                         commit(&sh.o_done[1]);
                         commit(&sh.v_empty[vst]);
+                        if (j + 1 == U.nkv1 && nkv_next[1] > 0) {
+                            if (!issue_first_s(1, nkv_next[1], kc + U.nkv1, (uit + 1) & 1))
+                                break;
+                            early[1] = true;
+                        }
                         continue;
                     }
                     if (j < U.nkv0) {   // PV0(j)
@@ -582,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool fast = !HAS_BIAS && scale_log2 > 0.f;   // max over raw scores, fused scale
         uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
+        for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
             const Unit U = decode_unit<CAUSAL>(u, p);
             const int nkv = i ? U.nkv1 : U.nkv0;
             const int row = U.q0 + i * kBlockM + t;
@@ -776,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             return ok;
         };
-        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uit) {
+        for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
             const Unit U = decode_unit<CAUSAL>(u, p);
             for (int j = 0; ok && j < U.nkv1; ++j) {
                 for (int i = 0; i < 2; ++i) {
@@ -815,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // O_i is released as soon as its last chunk is in registers, together with the next
             // unit's first pv_ready arrival (iteration 0 needs no rescale), so the next unit's
             // PV_i(0) does not wait for the gate arithmetic and global stores.
-            const bool has_next = u + static_cast<int>(gridDim.x) < p.num_units;
+            const bool has_next = unit_at(uit + 1) < p.num_units;
             for (int i = 0; i < 2; ++i) {
                 const int row = U.q0 + i * kBlockM + t;
                 const bool row_ok = row < p.N;

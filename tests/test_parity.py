@@ -144,3 +144,12 @@ def test_head_grouped_order_with_partial_group():
     o_ref, l_ref = sdpa_rows(inp["q"], inp["k"], inp["v"], picks, causal=True, scale=w.scale)
     idx = tuple(np.array(x) for x in zip(*picks))
     assert_close_to_oracle(o.cpu()[idx], lse.cpu()[idx], o_ref, l_ref, torch.bfloat16, "grouped")
+
+
+@pytest.mark.parametrize("B", [8, 13])
+def test_several_waves_of_units(B):
+    """More 256-row units than CTAs: each CTA takes one unit per wave, alternate waves in
+    reverse order.  B=8 (192 units on 148 SMs) ends in a partial reversed wave, B=13
+    (312 units) in a partial forward one; every output row is compared."""
+    w = Workload("waves", B=B, H=8, N=768, d=64, dtype="fp16", causal=True, seed=40 + B)
+    _full_check(w)
