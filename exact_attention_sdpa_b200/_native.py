@@ -22,7 +22,7 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIM
 ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+EXPORTED = ("attn_fwd", "attn_fwd_host", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
             "attn_debug_inject_stall", "attn_version")
 
 
@@ -55,6 +55,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         P = ctypes.POINTER(AttnTensor)
         lib.attn_fwd.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd.restype = ctypes.c_int
+        lib.attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p,
+                                      P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
+        lib.attn_fwd_host.restype = ctypes.c_int
         lib.attn_status_string.argtypes = [ctypes.c_int]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_last_device_status.argtypes = [ctypes.c_void_p]
@@ -135,32 +138,66 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[t
     return out, lse
 
 
+class Staging:
+    """Device buffers for one end-to-end problem: the layout of each host tensor
+    (dtype, shape, strides) on the device.  Reusing one across calls of the same
+    shape avoids an allocation per call; two of them on two streams let one
+    call's copies run under the other's kernel."""
+
+    def __init__(self, q, k, v, bias=None, gate=None, device=None):
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+
+        def like(t):
+            return None if t is None else torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, device=dev)
+
+        self.q, self.k, self.v, self.bias, self.gate = (like(t) for t in (q, k, v, bias, gate))
+        self.out = like(q if q.is_contiguous() else q.contiguous())
+        self.lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+
+
+def attn_fwd_host_raw(q, k, v, bias, gate, causal: bool, scale: float, out, lse, staging: Staging,
+                      stream: int) -> int:
+    """Direct call of attn_fwd_host: host tensors in and out, device staging from ``staging``."""
+    lib = load_library()
+    hq, hk, hv, hb, hg, ho = (make_view(t) for t in (q, k, v, bias, gate, out))
+    dq, dk, dv, db, dg, do = (make_view(t) for t in (staging.q, staging.k, staging.v, staging.bias, staging.gate,
+                                                    staging.out))
+    return lib.attn_fwd_host(_ref(hq), _ref(hk), _ref(hv), _ref(hb), _ref(hg), int(bool(causal)), float(scale),
+                             _ref(ho), None if lse is None else lse.data_ptr(),
+                             _ref(dq), _ref(dk), _ref(dv), _ref(db), _ref(dg), _ref(do),
+                             None if lse is None else staging.lse.data_ptr(), stream)
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[torch.Tensor] = None,
         gate: Optional[torch.Tensor] = None, causal: bool = False, scale: Optional[float] = None,
         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-        device: Optional[torch.device] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """The end-to-end call: host (ideally pinned) tensors in, host tensors out.
+        device: Optional[torch.device] = None, staging: Optional[Staging] = None,
+        stream: Optional[torch.cuda.Stream] = None, sync: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The end-to-end call: host tensors in, host tensors out (through attn_fwd_host).
 
-    Copies the inputs to ``device`` (default: the current CUDA device), runs
-    the fused kernel, copies O and lse back into ``out``/``lse`` (pinned host
-    tensors, allocated when not given) and waits for them.  Device tensors are
-    accepted too; then nothing is staged and the device results are returned.
+    The inputs should be pinned (``tensor.pin_memory()``) for asynchronous
+    copies.  ``out``/``lse`` are the host destinations (pinned, allocated when
+    not given); ``staging`` holds the device buffers (allocated when not given).
+    Everything is enqueued on ``stream`` (default: the current stream); with
+    ``sync`` the call waits for it, else the results are valid once the stream
+    has reached the call.  Device tensors are accepted too; then nothing is
+    staged and the device results are returned.
     """
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     if q.is_cuda:
-        return attn_fwd(q, k, v, bias, gate, causal, scale, out, lse)
-
-    def stage(t):
-        return None if t is None else t.to(dev, non_blocking=True)
-
-    o, l = attn_fwd(stage(q), stage(k), stage(v), stage(bias), stage(gate), causal, scale)
+        return attn_fwd(q, k, v, bias, gate, causal, scale, out, lse, stream)
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if staging is None:
+        staging = Staging(q, k, v, bias, gate, dev)
     if out is None:
-        out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        out = torch.empty(staging.out.shape, dtype=q.dtype, pin_memory=True)
     if lse is None:
-        lse = torch.empty(l.shape, dtype=l.dtype, pin_memory=True)
-    out.copy_(o, non_blocking=True)
-    lse.copy_(l, non_blocking=True)
-    torch.cuda.current_stream(dev).synchronize()
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, pin_memory=True)
+    st = stream or torch.cuda.current_stream(dev)
+    _check(attn_fwd_host_raw(q, k, v, bias, gate, causal, scale, out, lse, staging, st.cuda_stream))
+    if sync:
+        st.synchronize()
     return out, lse
 
 

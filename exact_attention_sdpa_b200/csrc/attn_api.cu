@@ -163,7 +163,11 @@ struct Maps {
 template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE>
 cudaError_t launch_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
     auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE>;
-    constexpr int smem = attn::BiasCfg<D, BIAS>::kDynBytes;
+    // At least 116 KB of dynamic shared memory, so that two CTAs (of two kernels running
+    // concurrently on different streams) never share an SM: each CTA allocates all 512
+    // tensor-memory columns, and a second one would only wait for the first to finish.
+    constexpr int smem = attn::BiasCfg<D, BIAS>::kDynBytes > 116 * 1024 ? attn::BiasCfg<D, BIAS>::kDynBytes
+                                                                      : 116 * 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int sms = sm_count();
@@ -216,13 +220,12 @@ unsigned int* status_word_ptr() {
     return ptrs[dev];
 }
 
-}  // namespace
-
-extern "C" {
-
-attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
-                       const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
-                       attn_tensor_t* out, float* lse, cudaStream_t stream) {
+// Every host-side check of attn_fwd, in its documented order; sets *empty for a
+// problem with B, H or N equal to 0 (valid, nothing to do).
+attn_status_t validate_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                           const attn_tensor_t* bias, const attn_tensor_t* gate, float scale,
+                           const attn_tensor_t* out, const float* lse, bool* empty) {
+    *empty = false;
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
     // dtype rules first: fp32 is a valid request this fused kernel does not serve
     if (q->dtype == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
@@ -236,6 +239,7 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     if (q->ndim == 4 && (q->shape[0] == 0 || q->shape[1] == 0 || q->shape[2] == 0)) {
         if (k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return ATTN_ERR_INVALID_ARG;
         if (!same_shape(q, k) || !same_shape(q, v) || !same_shape(q, out)) return ATTN_ERR_INVALID_ARG;
+        *empty = true;
         return ATTN_OK;
     }
     attn_status_t st;
@@ -266,6 +270,31 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     if (overlaps(out, q) || overlaps(out, k) || overlaps(out, v) || overlaps(out, bias) || overlaps(out, gate))
         return ATTN_ERR_INVALID_ARG;
     if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+
+    return ATTN_OK;
+}
+
+// A host view and its device staging view: same dtype, rank, shape and strides.
+bool same_layout(const attn_tensor_t* a, const attn_tensor_t* b) {
+    if ((a == nullptr) != (b == nullptr)) return false;
+    if (a == nullptr) return true;
+    if (a->dtype != b->dtype || !same_shape(a, b)) return false;
+    for (int i = 0; i < a->ndim; ++i)
+        if (a->stride[i] != b->stride[i]) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                       attn_tensor_t* out, float* lse, cudaStream_t stream) {
+    bool empty = false;
+    const attn_status_t st = validate_fwd(q, k, v, bias, gate, scale, out, lse, &empty);
+    if (st != ATTN_OK || empty) return st;
+    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], d = q->shape[3];
 
     // ---- launch
     Maps maps;
@@ -333,6 +362,48 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
         e = launch_dtype<__half>(static_cast<int>(d), causal != 0, bias != nullptr, gate != nullptr, maps, p,
                                  stream);
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                            const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                            attn_tensor_t* out, float* lse,
+                            const attn_tensor_t* q_dev, const attn_tensor_t* k_dev, const attn_tensor_t* v_dev,
+                            const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
+                            attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream) {
+    // every check before the first copy is enqueued
+    if (q_dev == nullptr || k_dev == nullptr || v_dev == nullptr || out_dev == nullptr) return ATTN_ERR_INVALID_ARG;
+    bool empty = false;
+    attn_status_t st = validate_fwd(q_dev, k_dev, v_dev, bias_dev, gate_dev, scale, out_dev, lse_dev, &empty);
+    if (st != ATTN_OK) return st;
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (!same_layout(q, q_dev) || !same_layout(k, k_dev) || !same_layout(v, v_dev) || !same_layout(out, out_dev) ||
+        !same_layout(bias, bias_dev) || !same_layout(gate, gate_dev))
+        return ATTN_ERR_INVALID_ARG;
+    if ((lse == nullptr) != (lse_dev == nullptr)) return ATTN_ERR_INVALID_ARG;
+    if (empty) return ATTN_OK;
+    const attn_tensor_t* hosts[6] = {q, k, v, out, bias, gate};
+    for (const attn_tensor_t* t : hosts)
+        if (t != nullptr && t->data == nullptr) return ATTN_ERR_INVALID_ARG;
+
+    // host -> device, one copy per input (the span from the first to one past the last element)
+    const attn_tensor_t* ins[5][2] = {{q, q_dev}, {k, k_dev}, {v, v_dev}, {bias, bias_dev}, {gate, gate_dev}};
+    for (auto& io : ins) {
+        if (io[0] == nullptr) continue;
+        if (cudaMemcpyAsync(io[1]->data, io[0]->data, static_cast<size_t>(span_bytes(io[0])),
+                            cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+    }
+    st = attn_fwd(q_dev, k_dev, v_dev, bias_dev, gate_dev, causal, scale, out_dev, lse_dev, stream);
+    if (st != ATTN_OK) return st;
+    // device -> host: O, then lse
+    if (cudaMemcpyAsync(out->data, out_dev->data, static_cast<size_t>(span_bytes(out)), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (lse != nullptr) {
+        const size_t n = static_cast<size_t>(q->shape[0] * q->shape[1] * q->shape[2]) * sizeof(float);
+        if (cudaMemcpyAsync(lse, lse_dev, n, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
 }
 
 const char* attn_status_string(attn_status_t status) {

@@ -96,6 +96,38 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
                        attn_tensor_t* out, float* lse,
                        cudaStream_t stream);
 
+/*
+ * attn_fwd_host -- the same operation end to end from HOST memory.
+ *
+ *   q, k, v, bias?, gate?   views of the inputs in host memory (layout rules of
+ *                           attn_fwd, except that they need not be device memory)
+ *   out, lse?               host destinations of O and lse (lse: B*H*N fp32)
+ *   q_dev ... out_dev, lse_dev
+ *                           caller-owned DEVICE staging buffers: each view has the
+ *                           dtype, shape and strides of its host counterpart; bias_dev
+ *                           / gate_dev / lse_dev are NULL exactly when bias / gate /
+ *                           lse are.
+ *
+ * Enqueued on `stream`, in order: one cudaMemcpyAsync per input (the span from
+ * its first to one past its last element) host -> device, attn_fwd on the
+ * staging views, then O and lse device -> host.  Returns once all of it is
+ * enqueued; the host results are valid once `stream` reaches the end of the
+ * call.  Host buffers should be page-locked (cudaHostAlloc, cudaHostRegister)
+ * so that the copies are asynchronous: calls on separate streams with separate
+ * staging buffers then run one problem's copies under another's kernel.  The
+ * library allocates nothing.  Errors: every check of attn_fwd applies to the
+ * staging views, a host view whose dtype, shape or strides differ from its
+ * staging view (or a NULL that does not match) is ATTN_ERR_INVALID_ARG, all
+ * before any copy is enqueued; ATTN_ERR_CUDA if a copy or the launch fails
+ * (earlier copies of the call may then already be enqueued).
+ */
+attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                            const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                            attn_tensor_t* out, float* lse,
+                            const attn_tensor_t* q_dev, const attn_tensor_t* k_dev, const attn_tensor_t* v_dev,
+                            const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
+                            attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream);
+
 /* A static, NUL-terminated description of a status code (never NULL). */
 const char* attn_status_string(attn_status_t status);
 

@@ -184,3 +184,59 @@ def test_product_path_does_not_reach_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not pat.search(text), fn
+
+
+# ---- attn_fwd_host: every check happens before the first copy is enqueued, so
+# CPU tensors stand in for both the host buffers and the device staging here.
+
+class _FakeStaging:
+    def __init__(self, q, k, v, bias=None, gate=None, out=None):
+        self.q, self.k, self.v, self.bias, self.gate = q, k, v, bias, gate
+        self.out = torch.zeros_like(q) if out is None else out
+        self.lse = torch.zeros(q.shape[:-1], dtype=torch.float32)
+
+
+def call_host(hq, hk, hv, ho, st, bias=None, gate=None, lse=None, scale=0.125):
+    return nat.attn_fwd_host_raw(hq, hk, hv, bias, gate, False, scale, ho, lse, st, 0)
+
+
+def test_host_entry_rejects_layout_mismatch(lib):
+    q, k, v, o = _qkv()
+    st = _FakeStaging(*_qkv()[:3])
+    assert call_host(q, k, v, o, _FakeStaging(*_qkv(N=32)[:3])) == nat.ATTN_ERR_INVALID_ARG      # shapes
+    padded = torch.zeros(1, 2, 64, 72, dtype=torch.float16)[..., :64]
+    assert call_host(q, k, v, o, _FakeStaging(padded, *_qkv()[1:3])) == nat.ATTN_ERR_INVALID_ARG  # strides
+    assert call_host(q, k, v, o, _FakeStaging(q.to(torch.bfloat16), *_qkv()[1:3])) != nat.ATTN_OK  # dtype
+    bias = torch.zeros(2, 64, 64, dtype=torch.float16)
+    assert call_host(q, k, v, o, st, bias=bias) == nat.ATTN_ERR_INVALID_ARG                        # bias vs none
+    st_b = _FakeStaging(*_qkv()[:3], bias=torch.zeros(2, 64, 64, dtype=torch.float16))
+    assert call_host(q, k, v, o, st_b) == nat.ATTN_ERR_INVALID_ARG                                 # none vs bias
+    assert call_host(q, k, v, torch.zeros(1, 2, 64, 32, dtype=torch.float16), st) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_host_entry_applies_device_checks_and_null_rules(lib):
+    q, k, v, o = _qkv()
+    f32 = _FakeStaging(*_qkv(dtype=torch.float32)[:3])
+    assert call_host(*_qkv(dtype=torch.float32), f32) == nat.ATTN_ERR_UNSUPPORTED
+    st = _FakeStaging(*_qkv()[:3])
+    assert call_host(q, k, v, o, st, scale=float("nan")) == nat.ATTN_ERR_INVALID_ARG
+    # lse on the host side without an lse staging buffer (and the reverse)
+    P = ctypes.POINTER(nat.AttnTensor)
+    views = [nat.make_view(t) for t in (q, k, v, o, st.q, st.k, st.v, st.out)]
+    refs = [ctypes.byref(x) for x in views]
+    lse = torch.zeros(1, 2, 64, dtype=torch.float32)
+    r = lib.attn_fwd_host(refs[0], refs[1], refs[2], None, None, 0, 0.1, refs[3], lse.data_ptr(),
+                          refs[4], refs[5], refs[6], None, None, refs[7], None, None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+    r = lib.attn_fwd_host(refs[0], refs[1], refs[2], None, None, 0, 0.1, refs[3], None,
+                          refs[4], refs[5], refs[6], None, None, refs[7], st.lse.data_ptr(), None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+    r = lib.attn_fwd_host(refs[0], refs[1], refs[2], None, None, 0, 0.1, refs[3], None,
+                          None, refs[5], refs[6], None, None, refs[7], None, None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_host_entry_empty_problem_is_ok(lib):
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
+    st = _FakeStaging(q.clone(), q.clone(), q.clone())
+    assert call_host(q, q.clone(), q.clone(), q.clone(), st) == nat.ATTN_OK
