@@ -102,6 +102,10 @@ struct Cfg {
     // d <= 64: P has columns of its own, so S_i(j+1) may be computed while the
     // softmax of S_i(j) runs; d = 128: P lives inside S_i (no room otherwise).
     static constexpr bool kSeparateP = (D <= 64);
+    // One exponential pair in kEmuPeriod goes through the FMA-pipe 2^x (0: none).  Measured
+    // on B200: at d=64 one in four beats one in three and none; at d=128 (MMA-bound) and
+    // d=32 (short units) the extra FMA-pipe work costs more than the MUFU time it saves.
+    static constexpr int kEmuPeriod = (D == 64) ? 4 : 0;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColP0 = (D == 128) ? 0 : 256;
     static constexpr uint32_t kColP1 = (D == 128) ? 128 : 320;
@@ -730,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
                 // p = 2^(x - m): x = s * scale_log2 on the fast path (s raw), x = y * log2(e) otherwise.
-                // One pair in three goes through the FMA-pipe exponential so that the
+                // At d=64 one pair in four goes through the FMA-pipe exponential so that the
                 // MUFU unit (16 lanes per clock per SM) is not the only exp resource.
                 const float xa = fast ? scale_log2 : kLog2e;
                 const float xb = -m_use;
@@ -743,7 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int pp = half * 32 + q2;
                         float x0, x1, e0, e1;
                         ffma2(x0, x1, s[2 * pp], s[2 * pp + 1], xa, xa, xb, xb);
-                        if (pp % 3 == 2) {
+                        constexpr int kEmu = Cfg<D>::kEmuPeriod;
+                        if (kEmu > 0 && pp % (kEmu > 0 ? kEmu : 1) == kEmu - 1) {
                             ex2_emu2(e0, e1, x0, x1);
                         } else {
                             e0 = ex2_approx(x0);
