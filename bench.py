@@ -18,6 +18,7 @@ import statistics
 import sys
 import threading
 import time
+from typing import Optional
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -109,26 +110,40 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: Optional[str] = None):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).  The process group
+    carries only the barrier and the max-over-ranks timing: replicas exchange no data.
+    NCCL on GPUs; gloo where no GPU is present (the CPU tests of this host logic)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
 def dist_max(x: float, world: int) -> float:
+    """The maximum of x over all ranks (the slowest replica sets the job time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """All ranks' work (each replica runs the full workload) over the slowest rank's time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
 def barrier(world: int):
@@ -200,7 +215,7 @@ def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
     e1.record(streams[0])
     torch.cuda.synchronize()
     ms = dist_max(e0.elapsed_time(e1) / steps, world)
-    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_tflops(world, flops, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
             "api": "fwd() -> attn_fwd_host (C ABI, pinned host buffers), 2 streams"}
 
@@ -275,7 +290,7 @@ def main():
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     ms_per_step = dist_max(total_ms / args.steps, world)
     mean_launch_ms = statistics.mean(launch_ms)
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs in, host outputs back, every step
     e2e = None if args.no_e2e else run_e2e(args, w, inp_cpu, out, lse, stream, world, flops)
