@@ -19,7 +19,14 @@ exponentials shifted by it.  Readings of points the pages leave open:
 
 * the explicit ``scale`` multiplies Q K^T, and the additive bias enters after
   scaling: s = scale * q.k + bias;
-* causal: key j is visible to query i iff j <= i (square problems only);
+* causal: key j is visible to query i iff j <= i + (Nk - Nq).  For square
+  problems (Nq = Nk, every workload the pages size) this is j <= i.  With
+  fewer queries than keys the queries are read as the last Nq positions of the
+  Nk-long sequence (the KV-cache reading of inskillml Module 9's general
+  ``scaled_dot_product_attention`` use: a prefill chunk or a decode step
+  attends to everything before and including itself), so the alignment is at
+  the bottom right; with more queries than keys the first Nq - Nk rows see no
+  key and are dead rows (below);
 * lse_i = m_i + ln(l_i) in natural log, of the scaled, biased, masked scores;
   the gate does not enter it;
 * the gate multiplies the normalised output elementwise by 1/(1+exp(-g));
@@ -57,19 +64,19 @@ def _bias_rows(bias: Optional[np.ndarray], b: int, h: int, rows: np.ndarray) -> 
     return bias[b, h, rows, :]                     # [B, H, Nq, Nk]
 
 
-def _attend_rows(qr, k, v, bias_r, gate_r, rows, causal, scale) -> Tuple[np.ndarray, np.ndarray]:
+def _attend_rows(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0) -> Tuple[np.ndarray, np.ndarray]:
     """Two-pass stable softmax attention for a block of query rows of one (b, h).
 
     qr: [r, d] queries; k, v: [Nk, d]; bias_r: [r, Nk] or None; rows: the
-    query indices of qr (for the causal mask).
+    query indices of qr (for the causal mask); offset = Nk - Nq.
     """
-    # step 1: scores s_ij = scale * q_i . k_j (+ bias_ij), causal keys j > i masked to -inf
+    # step 1: scores s_ij = scale * q_i . k_j (+ bias_ij), causal keys j > i + offset masked to -inf
     s = scale * (qr @ k.T)
     if bias_r is not None:
         s = s + bias_r
     if causal:
         keys = np.arange(k.shape[0])
-        s = np.where(keys[None, :] > rows[:, None], -np.inf, s)
+        s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
     # pass 1: row maximum
     m = s.max(axis=1)
     dead = ~np.isfinite(m) & (m < 0)               # every score of the row is -inf
@@ -91,8 +98,7 @@ def _attend_rows(qr, k, v, bias_r, gate_r, rows, causal, scale) -> Tuple[np.ndar
 def _check(q, k, v, causal):
     assert q.ndim == 4 and k.ndim == 4 and v.ndim == 4, "q, k, v must be [B, H, N, d]"
     assert k.shape == v.shape and q.shape[:2] == k.shape[:2] and q.shape[3] == k.shape[3]
-    if causal:
-        assert q.shape[2] == k.shape[2], "causal masking is defined here for Nq == Nk"
+    assert k.shape[2] >= 1, "at least one key"
 
 
 def sdpa_forward(q, k, v, bias=None, gate=None, causal: bool = False, scale: Optional[float] = None,
@@ -106,6 +112,7 @@ def sdpa_forward(q, k, v, bias=None, gate=None, causal: bool = False, scale: Opt
     q, k, v, bias, gate = (to_f64(t) for t in (q, k, v, bias, gate))
     _check(q, k, v, causal)
     B, H, Nq, d = q.shape
+    offset = k.shape[2] - Nq
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     O = np.zeros((B, H, Nq, d))
@@ -115,7 +122,7 @@ def sdpa_forward(q, k, v, bias=None, gate=None, causal: bool = False, scale: Opt
             for r0 in range(0, Nq, block_rows):
                 rows = np.arange(r0, min(Nq, r0 + block_rows))
                 o, lse = _attend_rows(q[b, h, rows], k[b, h], v[b, h], _bias_rows(bias, b, h, rows),
-                                      None if gate is None else gate[b, h, rows], rows, causal, scale)
+                                      None if gate is None else gate[b, h, rows], rows, causal, scale, offset)
                 O[b, h, rows] = o
                 L[b, h, rows] = lse
     return O, L
@@ -140,14 +147,12 @@ def sdpa_rows(q, k, v, picks: Sequence[Tuple[int, int, int]], bias=None, gate=No
         idx = np.array([i for _, i in lst])
         qr = to_f64(q[b, h][idx])
         kb, vb = to_f64(k[b, h]), to_f64(v[b, h])
-        if causal:
-            assert q.shape[2] == k.shape[2]
         br = None
         if bias is not None:
             bsel = bias[h] if bias.ndim == 3 else bias[b, h]
             br = to_f64(bsel[idx])
         gr = None if gate is None else to_f64(gate[b, h][idx])
-        o, lse = _attend_rows(qr, kb, vb, br, gr, idx, causal, scale)
+        o, lse = _attend_rows(qr, kb, vb, br, gr, idx, causal, scale, k.shape[2] - q.shape[2])
         for t, (n, _) in enumerate(lst):
             out_o[n] = o[t]
             out_l[n] = lse[t]

@@ -262,9 +262,52 @@ def pin_large_scores_stable(fwd):
     np.testing.assert_allclose(lse, lb, rtol=1e-14)
 
 
+def pin_causal_suffix_alignment(fwd):
+    # fewer queries than keys: the queries are the last Nq positions, so their rows must equal
+    # the last Nq rows of the square causal problem over the same keys (bottom-right alignment)
+    n, nq = 12, 5
+    q = _rand((2, 2, n, 6), 100)
+    k = _rand((2, 2, n, 6), 101)
+    v = _rand((2, 2, n, 6), 102)
+    bias = _rand((2, n, n), 103)
+    o_sq, l_sq = fwd(q, k, v, bias=bias, causal=True, scale=0.45)
+    o, lse = fwd(q[:, :, n - nq:], k, v, bias=bias[:, n - nq:], causal=True, scale=0.45)
+    np.testing.assert_allclose(o, o_sq[:, :, n - nq:], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, l_sq[:, :, n - nq:], rtol=0, atol=1e-14)
+
+
+def pin_decode_single_query(fwd):
+    # one query after all the keys sees every key: causal or not makes no difference
+    q = _rand((1, 3, 1, 8), 104)
+    k = _rand((1, 3, 9, 8), 105)
+    v = _rand((1, 3, 9, 8), 106)
+    o_c, l_c = fwd(q, k, v, causal=True, scale=0.3)
+    o_n, l_n = fwd(q, k, v, causal=False, scale=0.3)
+    np.testing.assert_allclose(o_c, o_n, rtol=0, atol=0)
+    np.testing.assert_allclose(l_c, l_n, rtol=0, atol=0)
+    ob, lb = _brute_force(q, k, v, None, None, False, 0.3)
+    np.testing.assert_allclose(o_c, ob, atol=1e-14)
+
+
+def pin_more_queries_than_keys(fwd):
+    # Nq > Nk, causal: the first Nq - Nk queries precede every key (dead rows: O = 0,
+    # lse = -inf); the others are the square problem on the last Nk queries
+    q = _rand((1, 2, 7, 4), 107)
+    k = _rand((1, 2, 4, 4), 108)
+    v = _rand((1, 2, 4, 4), 109)
+    o, lse = fwd(q, k, v, causal=True, scale=0.8)
+    assert np.all(o[:, :, :3] == 0.0) and np.all(lse[:, :, :3] == -np.inf)
+    o_sq, l_sq = fwd(q[:, :, 3:], k, v, causal=True, scale=0.8)
+    np.testing.assert_allclose(o[:, :, 3:], o_sq, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[:, :, 3:], l_sq, rtol=0, atol=1e-15)
+    ob, lb = _brute_force(q[:, :, 3:], k, v, None, None, True, 0.8)
+    np.testing.assert_allclose(o_sq, ob, atol=1e-14)
+
+
 PINS = [pin_hand_2x2, pin_hand_causal, pin_rows_sum_to_one, pin_identical_v_rows, pin_dominant_key,
         pin_causal_row0, pin_scale_zero_closed_form, pin_bias_shift, pin_key_permutation, pin_gate,
-        pin_brute_force, pin_torch_sdpa, pin_online_equals_two_pass, pin_large_scores_stable]
+        pin_brute_force, pin_torch_sdpa, pin_online_equals_two_pass, pin_large_scores_stable,
+        pin_causal_suffix_alignment, pin_decode_single_query, pin_more_queries_than_keys]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -333,7 +376,7 @@ def test_exact_upcast_of_half_inputs():
 def _mutant(kind):
     real = osdpa._attend_rows
 
-    def attend(qr, k, v, bias_r, gate_r, rows, causal, scale):
+    def attend(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0):
         if kind == "no_scale":
             scale = 1.0
         if kind == "bias_sign" and bias_r is not None:
@@ -342,7 +385,7 @@ def _mutant(kind):
             # reveal key i+1 as well (j <= i+1 instead of j <= i)
             keys = np.arange(k.shape[0])
             s = scale * (qr @ k.T) + (0 if bias_r is None else bias_r)
-            s = np.where(keys[None, :] > rows[:, None] + 1, -np.inf, s)
+            s = np.where(keys[None, :] > rows[:, None] + offset + 1, -np.inf, s)
             m = s.max(1)
             w = np.exp(s - m[:, None])
             o = (w @ v) / w.sum(1)[:, None]
@@ -355,7 +398,7 @@ def _mutant(kind):
             s = scale * (qr @ k.T) + (0 if bias_r is None else bias_r)
             if causal:
                 keys = np.arange(k.shape[0])
-                s = np.where(keys[None, :] > rows[:, None], -np.inf, s)
+                s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
             with np.errstate(over="ignore", invalid="ignore"):
                 w = np.exp(s)
                 o = (w @ v) / w.sum(1)[:, None]
@@ -364,20 +407,23 @@ def _mutant(kind):
                 o = o / (1 + np.exp(-gate_r))
             return o, lse
         if kind == "lse_log2":
-            o, lse = real(qr, k, v, bias_r, gate_r, rows, causal, scale)
+            o, lse = real(qr, k, v, bias_r, gate_r, rows, causal, scale, offset)
             return o, lse / math.log(2.0)
         if kind == "gate_not_sigmoid" and gate_r is not None:
-            o, lse = real(qr, k, v, bias_r, None, rows, causal, scale)
+            o, lse = real(qr, k, v, bias_r, None, rows, causal, scale, offset)
             return o * gate_r, lse
         if kind == "transposed_q":
             qr = qr[::-1]
-        return real(qr, k, v, bias_r, gate_r, rows, causal, scale)
+        if kind == "top_left_alignment":
+            offset = 0
+        return real(qr, k, v, bias_r, gate_r, rows, causal, scale, offset)
 
     return attend
 
 
 @pytest.mark.parametrize("kind", ["no_scale", "bias_sign", "causal_off_by_one", "k_for_v",
-                                  "no_max_shift", "lse_log2", "gate_not_sigmoid", "transposed_q"])
+                                  "no_max_shift", "lse_log2", "gate_not_sigmoid", "transposed_q",
+                                  "top_left_alignment"])
 def test_pins_catch_planted_mistake(kind, monkeypatch):
     monkeypatch.setattr(osdpa, "_attend_rows", _mutant(kind))
     caught = 0
