@@ -62,6 +62,12 @@ bool same_shape(const attn_tensor_t* a, const attn_tensor_t* b) {
     return true;
 }
 
+// Queries and keys: same batch, heads and head dim (the row counts may differ).
+bool same_bhd(const attn_tensor_t* q, const attn_tensor_t* k) {
+    return q->ndim == 4 && k->ndim == 4 && q->shape[0] == k->shape[0] && q->shape[1] == k->shape[1] &&
+           q->shape[3] == k->shape[3];
+}
+
 // ---------------------------------------------------------------------------
 // tensor maps (driver entry point fetched through the runtime, so the library
 // does not link libcuda directly)
@@ -112,13 +118,15 @@ bool encode_bias_map(CUtensorMap* map, const attn_tensor_t* b) {
     if (enc == nullptr) return false;
     const bool has_b = b->ndim == 4;
     const int64_t H = has_b ? b->shape[1] : b->shape[0];
-    const int64_t N = has_b ? b->shape[2] : b->shape[1];
+    const int64_t Nq = has_b ? b->shape[2] : b->shape[1];      // rows (queries)
+    const int64_t Nk = has_b ? b->shape[3] : b->shape[2];      // columns (keys)
     const int64_t si = has_b ? b->stride[2] : b->stride[1];
     const int64_t sh = has_b ? b->stride[1] : b->stride[0];
-    const int64_t row = N > 1 ? si : 8;
-    const int64_t head = H > 1 ? sh : row * N;
+    // strides of extent-1 dimensions are free; give them valid (16-byte multiple) values
+    const int64_t row = Nq > 1 ? si : (Nk + 7) / 8 * 8;
+    const int64_t head = H > 1 ? sh : row * Nq;
     const int64_t batch = (has_b && b->shape[0] > 1) ? b->stride[0] : head * H;
-    const cuuint64_t dims[4] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)(has_b ? b->shape[0] : 1)};
+    const cuuint64_t dims[4] = {(cuuint64_t)Nk, (cuuint64_t)Nq, (cuuint64_t)H, (cuuint64_t)(has_b ? b->shape[0] : 1)};
     const cuuint64_t strides[3] = {(cuuint64_t)(row * 2), (cuuint64_t)(head * 2), (cuuint64_t)(batch * 2)};
     const cuuint32_t box[4] = {64u, 128u, 1u, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
@@ -235,22 +243,22 @@ attn_status_t validate_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const
     if (gate != nullptr && gate->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
     if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
 
-    // empty problems: nothing to do
+    // empty problems (B, H or the query count 0): nothing to do
     if (q->ndim == 4 && (q->shape[0] == 0 || q->shape[1] == 0 || q->shape[2] == 0)) {
         if (k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return ATTN_ERR_INVALID_ARG;
-        if (!same_shape(q, k) || !same_shape(q, v) || !same_shape(q, out)) return ATTN_ERR_INVALID_ARG;
+        if (!same_shape(k, v) || !same_shape(q, out) || !same_bhd(q, k)) return ATTN_ERR_INVALID_ARG;
         *empty = true;
         return ATTN_OK;
     }
     attn_status_t st;
     if ((st = check_tensor(q, 4)) != ATTN_OK) return st;
-    if ((st = check_tensor(k, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(k, 4)) != ATTN_OK) return st;   // (a key count of 0 fails here)
     if ((st = check_tensor(v, 4)) != ATTN_OK) return st;
     if ((st = check_tensor(out, 4)) != ATTN_OK) return st;
-    if (!same_shape(q, k) || !same_shape(q, v) || !same_shape(q, out)) return ATTN_ERR_INVALID_ARG;
-    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], d = q->shape[3];
+    if (!same_shape(k, v) || !same_shape(q, out) || !same_bhd(q, k)) return ATTN_ERR_INVALID_ARG;
+    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
     if (d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (N > (int64_t(1) << 30) || B * H > (int64_t(1) << 24)) return ATTN_ERR_UNSUPPORTED;
+    if (N > (int64_t(1) << 30) || Nk > (int64_t(1) << 30) || B * H > (int64_t(1) << 24)) return ATTN_ERR_UNSUPPORTED;
     if (gate != nullptr) {
         if ((st = check_tensor(gate, 4)) != ATTN_OK) return st;
         if (!same_shape(q, gate)) return ATTN_ERR_INVALID_ARG;
@@ -258,10 +266,10 @@ attn_status_t validate_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const
     if (bias != nullptr) {
         if (bias->ndim == 3) {
             if ((st = check_tensor(bias, 3)) != ATTN_OK) return st;
-            if (bias->shape[0] != H || bias->shape[1] != N || bias->shape[2] != N) return ATTN_ERR_INVALID_ARG;
+            if (bias->shape[0] != H || bias->shape[1] != N || bias->shape[2] != Nk) return ATTN_ERR_INVALID_ARG;
         } else if (bias->ndim == 4) {
             if ((st = check_tensor(bias, 4)) != ATTN_OK) return st;
-            if (bias->shape[0] != B || bias->shape[1] != H || bias->shape[2] != N || bias->shape[3] != N)
+            if (bias->shape[0] != B || bias->shape[1] != H || bias->shape[2] != N || bias->shape[3] != Nk)
                 return ATTN_ERR_INVALID_ARG;
         } else {
             return ATTN_ERR_INVALID_ARG;
@@ -294,7 +302,7 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     bool empty = false;
     const attn_status_t st = validate_fwd(q, k, v, bias, gate, scale, out, lse, &empty);
     if (st != ATTN_OK || empty) return st;
-    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], d = q->shape[3];
+    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
 
     // ---- launch
     Maps maps;
@@ -311,8 +319,10 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     p.B = static_cast<int>(B);
     p.H = static_cast<int>(H);
     p.N = static_cast<int>(N);
+    p.Nk = static_cast<int>(Nk);
+    p.causal_off = static_cast<int>(Nk - N);
     p.num_q_pairs = static_cast<int>((N + attn::kRowsPerUnit - 1) / attn::kRowsPerUnit);
-    p.n_kv_tiles = static_cast<int>((N + attn::kBlockN - 1) / attn::kBlockN);
+    p.n_kv_tiles = static_cast<int>((Nk + attn::kBlockN - 1) / attn::kBlockN);
     const int64_t units = static_cast<int64_t>(p.num_q_pairs) * B * H;
     if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
     p.num_units = static_cast<int>(units);
@@ -321,7 +331,7 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     // unit order: when the K/V of all heads exceed the L2, schedule a few heads at a
     // time (enough query pairs to occupy every SM), else all heads together
     {
-        const double kv_bytes = 2.0 * static_cast<double>(B * H) * static_cast<double>(N) * d * 2.0;
+        const double kv_bytes = 2.0 * static_cast<double>(B * H) * static_cast<double>(Nk) * d * 2.0;
         const int sms = sm_count();
         int g = static_cast<int>(B * H);
         if (sms > 0 && kv_bytes > static_cast<double>(l2_bytes())) g = (sms + p.num_q_pairs - 1) / p.num_q_pairs;

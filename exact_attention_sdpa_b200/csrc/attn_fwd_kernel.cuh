@@ -65,10 +65,12 @@ constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned long long kDrainLimit = 1ull << 32;
 
 struct FwdParams {
-    int B, H, N;
+    int B, H, N;               // N: query rows
+    int Nk;                    // key rows
+    int causal_off;            // Nk - N: query i sees key j iff j <= i + causal_off (causal)
     int num_q_pairs;           // ceil(N / 256)
     int num_units;             // num_q_pairs * B * H
-    int n_kv_tiles;            // ceil(N / 128)
+    int n_kv_tiles;            // ceil(Nk / 128)
     int head_group;            // heads per scheduling group (see decode_unit)
     float scale;               // multiplies Q K^T
     float scale_log2;          // scale * log2(e)
@@ -268,8 +270,11 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
     U.h = U.bh % p.H;
     U.q0 = U.qp * kRowsPerUnit;
     if (CAUSAL) {
-        U.nkv0 = min(p.n_kv_tiles, 2 * U.qp + 1);
-        U.nkv1 = min(p.n_kv_tiles, 2 * U.qp + 2);
+        // key tiles up to the one holding the last visible key of the tile's last row; at
+        // least one (a tile whose rows all precede every key is processed once, fully masked)
+        const int last0 = U.q0 + kBlockM - 1 + p.causal_off, last1 = last0 + kBlockM;
+        U.nkv0 = last0 < 0 ? 1 : min(p.n_kv_tiles, last0 / kBlockN + 1);
+        U.nkv1 = last1 < 0 ? 1 : min(p.n_kv_tiles, last1 / kBlockN + 1);
     } else {
         U.nkv0 = U.nkv1 = p.n_kv_tiles;
     }
@@ -624,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Unit U = decode_unit<CAUSAL>(u, p);
             const int nkv = i ? U.nkv1 : U.nkv0;
             const int row = U.q0 + i * kBlockM + t;
-            const int diag = 2 * U.qp + i;          // the key tile holding this tile's diagonal
+            const int first_row = U.q0 + i * kBlockM;
             const T* bias_row = nullptr;
             if constexpr (HAS_BIAS)
                 bias_row = reinterpret_cast<const T*>(p.bias) + U.b * p.bias_sb + U.h * p.bias_sh +
@@ -656,11 +661,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 const int kv0 = j * kBlockN;
-                const bool need_mask = (kv0 + kBlockN > p.N) || (CAUSAL && j == diag);
+                // key tiles past the end, and (causal) tiles reaching past the first row's last key
+                const bool need_mask =
+                    (kv0 + kBlockN > p.Nk) || (CAUSAL && kv0 + kBlockN - 1 > first_row + p.causal_off);
                 float m_tile;   // tile maximum, log2 domain
                 if (fast) {
                     if (need_mask) {
-                        const int lim = CAUSAL ? min(p.N - kv0, row - kv0 + 1) : (p.N - kv0);
+                        const int lim = CAUSAL ? min(p.Nk - kv0, row + p.causal_off - kv0 + 1) : (p.Nk - kv0);
 #pragma unroll
                         for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
                     }
@@ -687,13 +694,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 // chunk (c % 64) / 8 of box c / 64, 128-byte swizzle
                                 raw = *reinterpret_cast<const uint4*>(
                                     brow + (c / 64) * BC::kBoxBytes + ((((c % 64) / 8) ^ (t & 7)) << 4));
-                            } else if (row < p.N && kv0 + c + 8 <= p.N) {
+                            } else if (row < p.N && kv0 + c + 8 <= p.Nk) {
                                 raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
                             } else {
                                 T e[8];
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
-                                    e[q] = (row < p.N && kv0 + c + q < p.N) ? bias_row[kv0 + c + q] : T(0.f);
+                                    e[q] = (row < p.N && kv0 + c + q < p.Nk) ? bias_row[kv0 + c + q] : T(0.f);
                                 raw = *reinterpret_cast<const uint4*>(e);
                             }
                             const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -714,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ++bcnt;
                     }
                     if (need_mask) {
-                        const int lim = CAUSAL ? min(p.N - kv0, row - kv0 + 1) : (p.N - kv0);
+                        const int lim = CAUSAL ? min(p.Nk - kv0, row + p.causal_off - kv0 + 1) : (p.Nk - kv0);
 #pragma unroll
                         for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
                     }

@@ -40,6 +40,11 @@ class Workload:
     bias: bool = False  # additive pair bias [H, N, N], shared over B
     gate: bool = False  # O <- sigmoid(G) * O, G has O's shape
     description: str = ""
+    Nk: Optional[int] = None   # key rows when they differ from the N query rows (KV-cache shapes)
+
+    @property
+    def n_keys(self) -> int:
+        return self.N if self.Nk is None else self.Nk
 
     @property
     def scale(self) -> float:
@@ -83,6 +88,7 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional[t
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed if seed is None else seed)
     shape = (w.B, w.H, w.N, w.d)
+    kv_shape = (w.B, w.H, w.n_keys, w.d)
     dt = w.torch_dtype
 
     def draw(*s):
@@ -92,24 +98,36 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional[t
         return x.to(dt)
 
     q = draw(*shape)
-    k = draw(*shape)
-    v = draw(*shape)
-    bias = draw(w.H, w.N, w.N) if w.bias else None
+    k = draw(*kv_shape)
+    v = draw(*kv_shape)
+    bias = draw(w.H, w.N, w.n_keys) if w.bias else None
     gate = draw(*shape) if w.gate else None
     return {"q": q, "k": k, "v": v, "bias": bias, "gate": gate}
 
 
 def attention_flops(w: Workload) -> float:
-    """The metric's FLOP count: 4*B*H*N^2*d, halved for causal."""
-    f = 4.0 * w.B * w.H * w.N * w.N * w.d
-    return f / 2.0 if w.causal else f
+    """The metric's FLOP count: 4*B*H*N^2*d, halved for causal (square problems).  With
+    Nk keys: 4*B*H*d times the number of visible (query, key) pairs, N*Nk without causal
+    masking, and with it the pairs j <= i + (Nk - N) (N*Nk - N*(N-1)/2 when N <= Nk)."""
+    if w.Nk is None:
+        f = 4.0 * w.B * w.H * w.N * w.N * w.d
+        return f / 2.0 if w.causal else f
+    n, nk = w.N, w.Nk
+    if not w.causal:
+        pairs = n * nk
+    else:
+        off = nk - n
+        pairs = sum(min(nk, max(0, i + off + 1)) for i in range(n))
+    return 4.0 * w.B * w.H * w.d * pairs
 
 
 def algorithmic_bytes(w: Workload) -> int:
     """Bytes one forward must move at least once: Q, K, V (and G, bias) read, O and lse written."""
     elem = 2
-    per_tensor = w.B * w.H * w.N * w.d * elem
-    n_tensors = 4 + (1 if w.gate else 0)          # q, k, v, o (+ gate)
-    bias = w.H * w.N * w.N * elem if w.bias else 0
+    per_q = w.B * w.H * w.N * w.d * elem
+    per_kv = w.B * w.H * w.n_keys * w.d * elem
+    per_tensor = per_q
+    n_tensors = 2 + (1 if w.gate else 0)          # q, o (+ gate); k, v below
+    bias = w.H * w.N * w.n_keys * elem if w.bias else 0
     lse = w.B * w.H * w.N * 4
-    return n_tensors * per_tensor + bias + lse
+    return n_tensors * per_tensor + 2 * per_kv + bias + lse

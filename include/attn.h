@@ -6,7 +6,7 @@
  * additive bias and sigmoid gate of the gated Evoformer variant named in the
  * gist.science FLASHLIGHT summary):
  *
- *     S   = scale * Q K^T (+ bias),   S_ij = -inf for j > i when causal
+ *     S   = scale * Q K^T (+ bias),   S_ij = -inf for j > i + (Nk - N) when causal
  *     O   = softmax_rows(S) V   (then O <- O * sigmoid(G) when a gate is given)
  *     lse = per-row natural-log logsumexp of S, i.e. m + ln(l) for the row
  *           maximum m and the sum l of exp(S - m); the gate does not enter it.
@@ -50,8 +50,8 @@ typedef enum {
 
 /*
  * A strided view of a device tensor.  shape and stride are in ELEMENTS, outer
- * to inner; only the first `ndim` entries are read.  Q, K, V, O and the gate
- * are 4-D [B, H, N, d]; the innermost stride must be 1 and every other stride
+ * to inner; only the first `ndim` entries are read.  Q, O and the gate are 4-D
+ * [B, H, N, d], K and V [B, H, Nk, d]; the innermost stride must be 1 and every other stride
  * times the element size must be a multiple of 16 bytes, and `data` must be
  * 16-byte aligned (tensor-memory-accelerator copies need both).
  */
@@ -66,14 +66,18 @@ typedef struct {
 /*
  * attn_fwd -- O = softmax(scale * Q K^T [+ bias]) V [* sigmoid(G)] and lse.
  *
- *   q       [B, H, N, d]  fp16 or bf16, device memory.
- *   k, v    [B, H, N, d]  same dtype, B, H, N and d as q.
- *   bias    nullable.  Additive score bias of q's dtype, either [H, N, N]
- *           (shared over B, the Evoformer pair bias) or [B, H, N, N]; the
+ *   q       [B, H, N, d]  fp16 or bf16, device memory: N query rows.
+ *   k, v    [B, H, Nk, d] same dtype, B, H and d as q; Nk >= 1 key rows (Nk may
+ *           differ from N: a prefill chunk or a decode step against a KV cache).
+ *   bias    nullable.  Additive score bias of q's dtype, either [H, N, Nk]
+ *           (shared over B, the Evoformer pair bias) or [B, H, N, Nk]; the
  *           innermost stride must be 1 and rows 16-byte aligned.
  *   gate    nullable.  [B, H, N, d] of q's dtype; O is multiplied elementwise
  *           by 1/(1+exp(-gate)) after normalisation.
- *   causal  nonzero: key j is visible to query i iff j <= i.
+ *   causal  nonzero: key j is visible to query i iff j <= i + (Nk - N), i.e. the
+ *           queries are the last N positions of the Nk-long sequence (bottom-right
+ *           alignment; j <= i when N == Nk).  With N > Nk the first N - Nk rows see
+ *           no key and get O = 0, lse = -inf.
  *   scale   multiplies Q K^T; must be finite (0 is legal).  Callers normally
  *           pass 1/sqrt(d).
  *   out     [B, H, N, d] of q's dtype, written (fp32 accumulator rounded to
@@ -82,8 +86,9 @@ typedef struct {
  *           natural log.  A row with every score -inf gets O = 0, lse = -inf.
  *   stream  CUDA stream of the launch (0 = legacy default stream).
  *
- * Supported: d in {32, 64, 128}; N >= 1 (any N, ragged tails are masked);
- * B*H >= 1.  N == 0 or B*H == 0 returns ATTN_OK without launching.
+ * Supported: d in {32, 64, 128}; N, Nk >= 1 (any sizes, ragged tails are
+ * masked); B*H >= 1.  N == 0 or B*H == 0 returns ATTN_OK without launching;
+ * Nk == 0 with N > 0 is ATTN_ERR_INVALID_ARG.
  * Errors are detected on the host before any launch and return a status with
  * no side effect: ATTN_ERR_INVALID_ARG for nulls, rank/shape/stride mismatch,
  * misalignment, aliasing of out with an input, or a non-finite scale;

@@ -240,3 +240,18 @@ def test_host_entry_empty_problem_is_ok(lib):
     q = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
     st = _FakeStaging(q.clone(), q.clone(), q.clone())
     assert call_host(q, q.clone(), q.clone(), q.clone(), st) == nat.ATTN_OK
+
+
+def test_rectangular_shape_rules(lib):
+    q = torch.zeros(1, 2, 48, 64, dtype=torch.float16)
+    o = torch.zeros_like(q)
+    k = torch.zeros(1, 2, 80, 64, dtype=torch.float16)
+    v80, v64 = torch.zeros_like(k), torch.zeros(1, 2, 64, 64, dtype=torch.float16)
+    assert call(q, k, v64, o) == nat.ATTN_ERR_INVALID_ARG                       # K and V key counts differ
+    assert call(q, k, v80, torch.zeros(1, 2, 80, 64, dtype=torch.float16)) == nat.ATTN_ERR_INVALID_ARG  # O not Q's shape
+    assert call(q, k, v80, o, bias=torch.zeros(2, 48, 48, dtype=torch.float16)) == nat.ATTN_ERR_INVALID_ARG
+    assert call(q, k, v80, o, bias=torch.zeros(2, 80, 80, dtype=torch.float16)) == nat.ATTN_ERR_INVALID_ARG
+    k32 = torch.zeros(1, 2, 80, 32, dtype=torch.float16)
+    assert call(q, k32, torch.zeros_like(k32), o) == nat.ATTN_ERR_INVALID_ARG    # head dims differ
+    k0 = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
+    assert call(q, k0, k0.clone(), o) == nat.ATTN_ERR_INVALID_ARG               # no keys for 48 queries

@@ -153,3 +153,33 @@ def test_several_waves_of_units(B):
     (312 units) in a partial forward one; every output row is compared."""
     w = Workload("waves", B=B, H=8, N=768, d=64, dtype="fp16", causal=True, seed=40 + B)
     _full_check(w)
+
+
+RECT = [  # (N query rows, Nk key rows, causal, d, dtype, bias, gate)
+    (128, 1024, True, 64, "fp16", False, False),      # prefill chunk against a KV cache
+    (1, 777, True, 128, "bf16", False, False),        # decode step
+    (3, 300, True, 64, "fp16", False, False),         # a few decode rows, ragged key tail
+    (300, 100, True, 64, "bf16", False, False),       # more queries than keys: 200 dead rows
+    (640, 2048, True, 64, "fp16", False, False),      # two and a half query pairs, offset 1408
+    (200, 513, False, 32, "bf16", True, True),        # non-causal with pair bias and gate
+    (257, 645, True, 32, "bf16", True, False),        # causal with bias, offset 388 (not a tile multiple)
+    (1000, 300, False, 128, "bf16", False, False),    # non-causal, Nq > Nk
+    (384, 500, True, 128, "fp16", True, True),        # d=128 bias path (global loads), offset 116
+]
+
+
+@pytest.mark.parametrize("N,Nk,causal,d,dtype,bias,gate", RECT)
+def test_rectangular_q_and_kv(N, Nk, causal, d, dtype, bias, gate):
+    """Nq != Nk: causal masking is aligned at the bottom right (query i sees keys
+    j <= i + Nk - Nq); every output row is compared with the oracle."""
+    w = Workload("rect", B=2, H=3, N=N, d=d, dtype=dtype, causal=causal, seed=60 + N % 17, Nk=Nk,
+                 bias=bias, gate=gate)
+    inp = make_inputs(w)
+    o, lse = _run(inp, w)
+    o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], bias=inp["bias"], gate=inp["gate"],
+                                causal=causal, scale=w.scale)
+    assert_close_to_oracle(o, lse, o_ref, l_ref, w.torch_dtype, f"rect{N}x{Nk}")
+    if causal and N > Nk:
+        dead = N - Nk
+        assert torch.all(o[:, :, :dead] == 0)
+        assert torch.all(torch.isneginf(lse[:, :, :dead]))
