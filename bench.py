@@ -172,7 +172,8 @@ def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
         dt = time.perf_counter() - t0
         if step >= warmup:
             secs += dt
-            vis = sum((i + 1) if w.causal else w.N for (_, _, i) in picks)
+            nk, off = w.n_keys, w.n_keys - w.N
+            vis = sum(min(nk, max(0, i + off + 1)) if w.causal else nk for (_, _, i) in picks)
             flops += 4.0 * w.d * vis
     cores = len(os.sched_getaffinity(0))
     sample = f"{rows_per_step} query rows (the last, i.e. heaviest) of one random (b,h) head per step, {steps} steps"
@@ -233,7 +234,8 @@ def main():
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     flops = attention_flops(w)
-    config = {"workload": w.name, "description": w.description, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+    config = {"workload": w.name, "description": w.description, "B": w.B, "H": w.H, "N": w.N, "Nk": w.n_keys,
+              "d": w.d,
               "causal": w.causal, "bias": w.bias, "gate": w.gate, "dtype": w.dtype,
               "inputs_bytes": algorithmic_bytes(w),
               "l2": "no flush: inputs+outputs larger than the 126 MB L2" if algorithmic_bytes(w) > 126e6

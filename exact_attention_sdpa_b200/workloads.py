@@ -74,6 +74,9 @@ WORKLOADS: Dict[str, Workload] = {
                  bias=True, gate=True,
                  description="Evoformer-style gated row attention, R=256 H=8 N=256 d=32 bf16, "
                              "pair bias [H,N,N], sigmoid gate"),
+        Workload("prefill_chunk", B=8, H=12, N=2048, d=64, dtype="fp16", causal=True, seed=5, Nk=8192,
+                 description="a 2048-row prefill chunk against an 8192-row KV cache, B=8 H=12 d=64 fp16, "
+                             "causal (bottom-right aligned)"),
     ]
 }
 

@@ -49,7 +49,7 @@ def _sampled_rows(w: Workload, n_bh=4, seed=0):
     return picks
 
 
-@pytest.mark.parametrize("name", ["n8192_causal", "long_wide"])
+@pytest.mark.parametrize("name", ["n8192_causal", "long_wide", "prefill_chunk"])
 def test_workload_full_size_sampled(name):
     """Full-size problems in the launch configuration the benchmark times;
     the oracle computes a sample of output rows one by one."""
