@@ -41,7 +41,7 @@ from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
-__all__ = ["sdpa_forward", "sdpa_rows", "to_f64"]
+__all__ = ["sdpa_forward", "sdpa_rows", "sdpa_backward", "to_f64"]
 
 
 def to_f64(x) -> Optional[np.ndarray]:
@@ -157,3 +157,66 @@ def sdpa_rows(q, k, v, picks: Sequence[Tuple[int, int, int]], bias=None, gate=No
             out_o[n] = o[t]
             out_l[n] = lse[t]
     return out_o, out_l
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+def _grad_rows(q, k, v, do, causal, scale, offset):
+    """Gradients of one (b, h) head without bias or gate, from the definition.
+
+    These are the derivatives of Equation (1) of aiinarabic.com
+    "flash-attention" (S = scale Q K^T, masked; P = softmax_rows(S); O = P V)
+    with respect to Q, K and V, given an upstream gradient dO.  (The same
+    page's recomputation section is why a fused backward rebuilds S and P from
+    Q, K and the saved normaliser; the oracle simply forms them.)
+
+        dV = P^T dO
+        dP = dO V^T
+        dS = P * (dP - rowsum(P * dP))        (softmax Jacobian, row by row)
+        dQ = scale dS K,   dK = scale dS^T Q
+
+    P is formed here with the two-pass softmax of the forward definition (not
+    from a saved lse), so the oracle does not depend on the forward under test.
+    """
+    s = scale * (q @ k.T)
+    if causal:
+        rows = np.arange(q.shape[0])
+        keys = np.arange(k.shape[0])
+        s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
+    m = s.max(axis=1)
+    dead = ~np.isfinite(m)
+    m_safe = np.where(dead, 0.0, m)
+    w = np.exp(s - m_safe[:, None])
+    l = w.sum(axis=1)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        p = w / l[:, None]
+    p = np.where(dead[:, None], 0.0, p)
+    dv = p.T @ do
+    dp = do @ v.T
+    ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv
+
+
+def sdpa_backward(q, k, v, do, causal: bool = False, scale: Optional[float] = None
+                  ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(dQ, dK, dV) in float64 for O = softmax(scale Q K^T [causal]) V and upstream dO.
+
+    q, do: [B,H,Nq,d]; k, v: [B,H,Nk,d]; causal masking aligned as in the forward
+    (key j visible to query i iff j <= i + Nk - Nq).  No bias or gate.
+    """
+    q, k, v, do = (to_f64(t) for t in (q, k, v, do))
+    _check(q, k, v, causal)
+    assert do.shape == q.shape
+    B, H, Nq, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dQ, dK, dV = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    for b in range(B):
+        for h in range(H):
+            dQ[b, h], dK[b, h], dV[b, h] = _grad_rows(q[b, h], k[b, h], v[b, h], do[b, h], causal, scale,
+                                                      k.shape[2] - Nq)
+    return dQ, dK, dV
