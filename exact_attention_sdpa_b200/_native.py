@@ -22,7 +22,7 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIM
 ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_fwd_host", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+EXPORTED = ("attn_fwd", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
             "attn_debug_inject_stall", "attn_version")
 
 
@@ -58,6 +58,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p,
                                       P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_host.restype = ctypes.c_int
+        lib.attn_bwd.argtypes = [P, P, P, P, ctypes.c_void_p, P, ctypes.c_int, ctypes.c_float, P, P, P,
+                                 ctypes.c_void_p]
+        lib.attn_bwd.restype = ctypes.c_int
         lib.attn_status_string.argtypes = [ctypes.c_int]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_last_device_status.argtypes = [ctypes.c_void_p]
@@ -136,6 +139,34 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[t
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
     _check(attn_fwd_raw(q, k, v, bias, gate, causal, scale, out, lse, s))
     return out, lse
+
+
+def attn_bwd_raw(q, k, v, out, lse, dout, causal: bool, scale: float, dq, dk, dv, stream: int) -> int:
+    """Direct call of attn_bwd with torch tensors; returns the status code."""
+    lib = load_library()
+    vq, vk, vv, vo, vdo, vdq, vdk, vdv = (make_view(t) for t in (q, k, v, out, dout, dq, dk, dv))
+    return lib.attn_bwd(_ref(vq), _ref(vk), _ref(vv), _ref(vo), None if lse is None else lse.data_ptr(), _ref(vdo),
+                        int(bool(causal)), float(scale), _ref(vdq), _ref(vdk), _ref(vdv), stream)
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+             dout: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(dQ, dK, dV) of attn_fwd (no bias or gate) for the upstream gradient ``dout``.
+
+    ``out`` and ``lse`` are attn_fwd's outputs for the same q, k, v, causal and
+    scale.  CUDA tensors; asynchronous on ``stream`` (default: the current one).
+    """
+    if not q.is_cuda:
+        raise ValueError("attn_bwd takes CUDA tensors")
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format)
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format)
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(attn_bwd_raw(q, k, v, out, lse, dout, causal, scale, dq, dk, dv, s))
+    return dq, dk, dv
 
 
 class Staging:

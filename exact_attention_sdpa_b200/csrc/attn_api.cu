@@ -10,6 +10,7 @@
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_bwd_kernel.cuh"
 
 namespace {
 
@@ -282,6 +283,34 @@ attn_status_t validate_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const
     return ATTN_OK;
 }
 
+// ---------------------------------------------------------------------------
+// backward launches
+// ---------------------------------------------------------------------------
+template <typename T, int D, bool CAUSAL>
+cudaError_t launch_bwd_t(const attn::bwd::BwdParams& p, cudaStream_t stream) {
+    constexpr int smem = attn::bwd::BwdSmem<D>::kBytes;
+    auto kdkdv = attn::bwd::attn_bwd_dkdv_kernel<T, D, CAUSAL>;
+    auto kdq = attn::bwd::attn_bwd_dq_kernel<T, D, CAUSAL>;
+    cudaError_t e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const dim3 g_kv((p.Nk + attn::bwd::kRows - 1) / attn::bwd::kRows, p.B * p.H);
+    const dim3 g_q((p.N + attn::bwd::kRows - 1) / attn::bwd::kRows, p.B * p.H);
+    kdkdv<<<g_kv, attn::bwd::kThreads, smem, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    kdq<<<g_q, attn::bwd::kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_bwd_dtype(int d, bool causal, const attn::bwd::BwdParams& p, cudaStream_t s) {
+    if (d == 32) return causal ? launch_bwd_t<T, 32, true>(p, s) : launch_bwd_t<T, 32, false>(p, s);
+    if (d == 64) return causal ? launch_bwd_t<T, 64, true>(p, s) : launch_bwd_t<T, 64, false>(p, s);
+    return causal ? launch_bwd_t<T, 128, true>(p, s) : launch_bwd_t<T, 128, false>(p, s);
+}
+
 // A host view and its device staging view: same dtype, rank, shape and strides.
 bool same_layout(const attn_tensor_t* a, const attn_tensor_t* b) {
     if ((a == nullptr) != (b == nullptr)) return false;
@@ -414,6 +443,57 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
         if (cudaMemcpyAsync(lse, lse_dev, n, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return ATTN_ERR_CUDA;
     }
     return ATTN_OK;
+}
+
+attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* out, const float* lse, const attn_tensor_t* dout, int causal,
+                       float scale, attn_tensor_t* dq, attn_tensor_t* dk, attn_tensor_t* dv,
+                       cudaStream_t stream) {
+    bool empty = false;
+    attn_status_t st = validate_fwd(q, k, v, nullptr, nullptr, scale, out, lse, &empty);
+    if (st != ATTN_OK) return st;
+    if (dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (dout->dtype != q->dtype || dq->dtype != q->dtype || dk->dtype != q->dtype || dv->dtype != q->dtype)
+        return ATTN_ERR_UNSUPPORTED;
+    if (!same_shape(dout, q) || !same_shape(dq, q) || !same_shape(dk, k) || !same_shape(dv, k))
+        return ATTN_ERR_INVALID_ARG;
+    if (empty) return ATTN_OK;
+    if (lse == nullptr) return ATTN_ERR_INVALID_ARG;
+    if ((st = check_tensor(dout, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(dq, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(dk, 4)) != ATTN_OK) return st;
+    if ((st = check_tensor(dv, 4)) != ATTN_OK) return st;
+    const attn_tensor_t* outs[3] = {dq, dk, dv};
+    const attn_tensor_t* ins[5] = {q, k, v, out, dout};
+    for (int a = 0; a < 3; ++a) {
+        for (int b = 0; b < 5; ++b)
+            if (overlaps(outs[a], ins[b])) return ATTN_ERR_INVALID_ARG;
+        for (int b = a + 1; b < 3; ++b)
+            if (overlaps(outs[a], outs[b])) return ATTN_ERR_INVALID_ARG;
+    }
+    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
+    if (B * H > 65535) return ATTN_ERR_UNSUPPORTED;
+
+    attn::bwd::BwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = static_cast<int>(B);
+    p.H = static_cast<int>(H);
+    p.N = static_cast<int>(N);
+    p.Nk = static_cast<int>(Nk);
+    p.causal_off = static_cast<int>(Nk - N);
+    p.scale = scale;
+    p.q = q->data; p.q_sb = q->stride[0]; p.q_sh = q->stride[1]; p.q_si = q->stride[2];
+    p.k = k->data; p.k_sb = k->stride[0]; p.k_sh = k->stride[1]; p.k_si = k->stride[2];
+    p.v = v->data; p.v_sb = v->stride[0]; p.v_sh = v->stride[1]; p.v_si = v->stride[2];
+    p.o = out->data; p.o_sb = out->stride[0]; p.o_sh = out->stride[1]; p.o_si = out->stride[2];
+    p.dout = dout->data; p.do_sb = dout->stride[0]; p.do_sh = dout->stride[1]; p.do_si = dout->stride[2];
+    p.lse = lse;
+    p.dq = dq->data; p.dq_sb = dq->stride[0]; p.dq_sh = dq->stride[1]; p.dq_si = dq->stride[2];
+    p.dk = dk->data; p.dk_sb = dk->stride[0]; p.dk_sh = dk->stride[1]; p.dk_si = dk->stride[2];
+    p.dv = dv->data; p.dv_sb = dv->stride[0]; p.dv_sh = dv->stride[1]; p.dv_si = dv->stride[2];
+    cudaError_t e = q->dtype == ATTN_BF16 ? launch_bwd_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, p, stream)
+                                          : launch_bwd_dtype<__half>(static_cast<int>(d), causal != 0, p, stream);
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 const char* attn_status_string(attn_status_t status) {

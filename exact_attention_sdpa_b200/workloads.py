@@ -23,7 +23,7 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "algorithmic_bytes"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_grad_output", "attention_flops", "algorithmic_bytes"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -134,3 +134,12 @@ def algorithmic_bytes(w: Workload) -> int:
     bias = w.H * w.N * w.n_keys * elem if w.bias else 0
     lse = w.B * w.H * w.N * 4
     return n_tensors * per_tensor + 2 * per_kv + bias + lse
+
+
+def make_grad_output(w: Workload, seed: Optional[int] = None) -> torch.Tensor:
+    """An upstream gradient dO for the backward: N(0,1) of O's shape in the workload's
+    dtype, from its own generator (seed + 1000 by default) so that the forward inputs
+    are the same bits with or without it."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed((w.seed if seed is None else seed) + 1000)
+    return torch.randn(w.B, w.H, w.N, w.d, generator=g, dtype=torch.float32).to(w.torch_dtype)

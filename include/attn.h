@@ -133,6 +133,34 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
                             const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
                             attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream);
 
+/*
+ * attn_bwd -- gradients of attn_fwd (without bias or gate) for an upstream dO:
+ *
+ *     P  = exp(scale Q K^T - lse)  (masked as in the forward)
+ *     dV = P^T dO,  dS = P * (dO V^T - D),  D_i = sum_c dO_ic O_ic
+ *     dQ = scale dS K,  dK = scale dS^T Q
+ *
+ * (the derivatives of the forward's definition; S and P are recomputed tile by
+ * tile from Q, K and the forward's lse, as the recomputation section of
+ * aiinarabic.com "flash-attention" describes, and never stored).
+ *
+ *   q, k, v, causal, scale   exactly as given to attn_fwd
+ *   out, lse                 attn_fwd's O [B, H, N, d] and lse (B*H*N fp32, required)
+ *   dout                     upstream gradient, O's shape and dtype
+ *   dq                       [B, H, N, d], written; dk, dv [B, H, Nk, d], written
+ *                            (fp32 accumulation, rounded to nearest-even into
+ *                            the dtype); none may overlap an input or another.
+ *
+ * Layout rules and errors as attn_fwd; additionally ATTN_ERR_INVALID_ARG for a
+ * missing lse, dout, dq, dk or dv, a shape mismatch or an overlap, and
+ * ATTN_ERR_UNSUPPORTED for B*H > 65535.  Asynchronous on `stream` (two kernel
+ * launches); allocates nothing.
+ */
+attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* out, const float* lse, const attn_tensor_t* dout, int causal,
+                       float scale, attn_tensor_t* dq, attn_tensor_t* dk, attn_tensor_t* dv,
+                       cudaStream_t stream);
+
 /* A static, NUL-terminated description of a status code (never NULL). */
 const char* attn_status_string(attn_status_t status);
 

@@ -255,3 +255,26 @@ def test_rectangular_shape_rules(lib):
     assert call(q, k32, torch.zeros_like(k32), o) == nat.ATTN_ERR_INVALID_ARG    # head dims differ
     k0 = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
     assert call(q, k0, k0.clone(), o) == nat.ATTN_ERR_INVALID_ARG               # no keys for 48 queries
+
+
+def test_backward_argument_checks(lib):
+    q, k, v, o = _qkv()
+    lse = torch.zeros(1, 2, 64, dtype=torch.float32)
+    do, dq, dk, dv = (torch.zeros_like(q) for _ in range(4))
+
+    def bwd(**kw):
+        a = dict(q=q, k=k, v=v, out=o, lse=lse, dout=do, dq=dq, dk=dk, dv=dv)
+        a.update(kw)
+        return nat.attn_bwd_raw(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], False, 0.125,
+                                a["dq"], a["dk"], a["dv"], 0)
+
+    assert bwd(lse=None) == nat.ATTN_ERR_INVALID_ARG
+    assert bwd(dq=torch.zeros(1, 2, 32, 64, dtype=torch.float16)) == nat.ATTN_ERR_INVALID_ARG
+    assert bwd(dk=q) == nat.ATTN_ERR_INVALID_ARG                                  # overlaps an input
+    assert bwd(dv=dk) == nat.ATTN_ERR_INVALID_ARG                                 # overlaps another output
+    assert bwd(dout=do.to(torch.bfloat16)) == nat.ATTN_ERR_UNSUPPORTED
+    q32 = torch.zeros(1, 2, 64, 64, dtype=torch.float32)
+    assert bwd(q=q32) == nat.ATTN_ERR_UNSUPPORTED
+    e = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
+    assert nat.attn_bwd_raw(e, k, v, e.clone(), None, e.clone(), False, 0.1, e.clone(), torch.zeros_like(k),
+                            torch.zeros_like(v), 0) == nat.ATTN_OK                 # no query rows: nothing to do
