@@ -221,6 +221,57 @@ def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
             "api": "fwd() -> attn_fwd_host (C ABI, pinned host buffers), 2 streams"}
 
 
+def fp32_fma_peak_tflops(sm_mhz: float) -> float:
+    """FP32 FMA peak of a B200: 148 SMs x 128 FP32 lanes x 2 FLOP per clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_bwd(args, w, config):
+    """The backward on one GPU: K timed attn_bwd launches (two kernels each) after W warm-ups,
+    inputs, O, lse and dO resident.  FLOPs: the usual 2.5x the forward's (five N x N x d
+    products against two); the kernels recompute S and dP per block, seven products in all."""
+    from exact_attention_sdpa_b200 import attn_bwd, attn_fwd, load_library
+    from exact_attention_sdpa_b200.workloads import make_grad_output
+    load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = {k: (None if t is None else t.to(dev)) for k, t in make_inputs(w).items()}
+    assert inp["bias"] is None and inp["gate"] is None, "the backward takes no bias or gate"
+    do = make_grad_output(w).to(dev)
+    out, lse = attn_fwd(inp["q"], inp["k"], inp["v"], causal=w.causal, scale=w.scale)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        attn_bwd(inp["q"], inp["k"], inp["v"], out, lse, do, causal=w.causal, scale=w.scale, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    flops = 2.5 * attention_flops(w)
+    value = flops / (ms * 1e-3) / 1e12
+    cs = clocks.summary()
+    peak = fp32_fma_peak_tflops(cs["sm_max_mhz"] or 1965.0)
+    line = {"metric": "attention bwd TFLOPS (2.5 x forward FLOPs)", "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs and dO)",
+            "config": dict(config, **{"pass": "backward"}),
+            "roofline": {"bound": "alu", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                         "peak_source": "FP32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock",
+                         "traffic": None, "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
+                         "algorithmic_flops_per_launch": flops},
+            "gpu_launches": 2 * steps, "e2e": None, "clocks": cs}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -231,6 +282,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-staged end-to-end leg (profiling runs)")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward (attn_bwd) on the workload instead of the forward")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     flops = attention_flops(w)
@@ -255,6 +308,8 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
+    if args.bwd:
+        return run_bwd(args, w, config)
     world, rank, local = dist_setup(args.gpus)
     from exact_attention_sdpa_b200 import attn_fwd, load_library
     load_library()
