@@ -30,7 +30,13 @@ exponentials shifted by it.  Readings of points the pages leave open:
 * lse_i = m_i + ln(l_i) in natural log, of the scaled, biased, masked scores;
   the gate does not enter it;
 * the gate multiplies the normalised output elementwise by 1/(1+exp(-g));
-* a row whose every score is -inf has O = 0 and lse = -inf.
+* a row whose every score is -inf has O = 0 and lse = -inf;
+* score modifications (inskillml Module 9's list of attention variants and
+  patterns; FLASHLIGHT's named variants), all optional and applied in this
+  order to s = scale * q.k + bias: ALiBi adds -slope_h * |i + (Nk - Nq) - j|
+  (a per-head linear distance penalty); a logit softcap c > 0 replaces s by
+  c * tanh(s / c); a left window w >= 0 masks keys j < i + (Nk - Nq) - w (a
+  sliding window, together with the causal mask a band of w + 1 keys).
 
 Inputs of any float dtype are upcast exactly to float64 before any arithmetic.
 Parity: pinned (see tests/test_oracle.py for the pins).
@@ -64,18 +70,29 @@ def _bias_rows(bias: Optional[np.ndarray], b: int, h: int, rows: np.ndarray) -> 
     return bias[b, h, rows, :]                     # [B, H, Nq, Nk]
 
 
-def _attend_rows(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0) -> Tuple[np.ndarray, np.ndarray]:
+def _attend_rows(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0, mods=None) -> Tuple[np.ndarray, np.ndarray]:
     """Two-pass stable softmax attention for a block of query rows of one (b, h).
 
     qr: [r, d] queries; k, v: [Nk, d]; bias_r: [r, Nk] or None; rows: the
-    query indices of qr (for the causal mask); offset = Nk - Nq.
+    query indices of qr (for the causal mask); offset = Nk - Nq; mods: None or
+    a dict with "alibi_slope" (this head's slope), "softcap", "window_left".
     """
     # step 1: scores s_ij = scale * q_i . k_j (+ bias_ij), causal keys j > i + offset masked to -inf
     s = scale * (qr @ k.T)
     if bias_r is not None:
         s = s + bias_r
+    keys = np.arange(k.shape[0])
+    if mods is not None:
+        slope = mods.get("alibi_slope")
+        if slope is not None:
+            s = s - slope * np.abs(rows[:, None] + offset - keys[None, :])
+        cap = mods.get("softcap", 0.0)
+        if cap and cap > 0:
+            s = cap * np.tanh(s / cap)
+        w = mods.get("window_left", -1)
+        if w is not None and w >= 0:
+            s = np.where(keys[None, :] < rows[:, None] + offset - w, -np.inf, s)
     if causal:
-        keys = np.arange(k.shape[0])
         s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
     # pass 1: row maximum
     m = s.max(axis=1)
@@ -101,14 +118,24 @@ def _check(q, k, v, causal):
     assert k.shape[2] >= 1, "at least one key"
 
 
+def _head_mods(softcap, alibi_slopes, window_left, h):
+    if not softcap and alibi_slopes is None and (window_left is None or window_left < 0):
+        return None
+    return {"softcap": softcap or 0.0, "window_left": -1 if window_left is None else window_left,
+            "alibi_slope": None if alibi_slopes is None else float(alibi_slopes[h])}
+
+
 def sdpa_forward(q, k, v, bias=None, gate=None, causal: bool = False, scale: Optional[float] = None,
-                 block_rows: int = 1024) -> Tuple[np.ndarray, np.ndarray]:
+                 block_rows: int = 1024, softcap: float = 0.0, alibi_slopes=None,
+                 window_left: int = -1) -> Tuple[np.ndarray, np.ndarray]:
     """Full forward: returns (O [B,H,Nq,d], lse [B,H,Nq]) in float64.
 
     q: [B,H,Nq,d]; k, v: [B,H,Nk,d]; bias: [H,Nq,Nk] or [B,H,Nq,Nk] or None;
-    gate: [B,H,Nq,d] or None; scale defaults to 1/sqrt(d).
+    gate: [B,H,Nq,d] or None; scale defaults to 1/sqrt(d); softcap, alibi_slopes
+    ([H]) and window_left as in the module docstring (off by default).
     Query rows are processed in blocks of ``block_rows`` only to bound memory.
     """
+    alibi_slopes = None if alibi_slopes is None else to_f64(alibi_slopes)
     q, k, v, bias, gate = (to_f64(t) for t in (q, k, v, bias, gate))
     _check(q, k, v, causal)
     B, H, Nq, d = q.shape
@@ -122,14 +149,16 @@ def sdpa_forward(q, k, v, bias=None, gate=None, causal: bool = False, scale: Opt
             for r0 in range(0, Nq, block_rows):
                 rows = np.arange(r0, min(Nq, r0 + block_rows))
                 o, lse = _attend_rows(q[b, h, rows], k[b, h], v[b, h], _bias_rows(bias, b, h, rows),
-                                      None if gate is None else gate[b, h, rows], rows, causal, scale, offset)
+                                      None if gate is None else gate[b, h, rows], rows, causal, scale, offset,
+                                      _head_mods(softcap, alibi_slopes, window_left, h))
                 O[b, h, rows] = o
                 L[b, h, rows] = lse
     return O, L
 
 
 def sdpa_rows(q, k, v, picks: Sequence[Tuple[int, int, int]], bias=None, gate=None, causal: bool = False,
-              scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+              scale: Optional[float] = None, softcap: float = 0.0, alibi_slopes=None,
+              window_left: int = -1) -> Tuple[np.ndarray, np.ndarray]:
     """Selected output rows only: picks = [(b, h, i), ...]; returns (O [n,d], lse [n]) in float64.
 
     Used to check full-size problems on a sample of rows; each row is computed
@@ -152,7 +181,9 @@ def sdpa_rows(q, k, v, picks: Sequence[Tuple[int, int, int]], bias=None, gate=No
             bsel = bias[h] if bias.ndim == 3 else bias[b, h]
             br = to_f64(bsel[idx])
         gr = None if gate is None else to_f64(gate[b, h][idx])
-        o, lse = _attend_rows(qr, kb, vb, br, gr, idx, causal, scale, k.shape[2] - q.shape[2])
+        slopes = None if alibi_slopes is None else to_f64(alibi_slopes)
+        o, lse = _attend_rows(qr, kb, vb, br, gr, idx, causal, scale, k.shape[2] - q.shape[2],
+                              _head_mods(softcap, slopes, window_left, h))
         for t, (n, _) in enumerate(lst):
             out_o[n] = o[t]
             out_l[n] = lse[t]

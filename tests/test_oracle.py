@@ -376,7 +376,7 @@ def test_exact_upcast_of_half_inputs():
 def _mutant(kind):
     real = osdpa._attend_rows
 
-    def attend(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0):
+    def attend(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0, mods=None):
         if kind == "no_scale":
             scale = 1.0
         if kind == "bias_sign" and bias_r is not None:
@@ -407,16 +407,16 @@ def _mutant(kind):
                 o = o / (1 + np.exp(-gate_r))
             return o, lse
         if kind == "lse_log2":
-            o, lse = real(qr, k, v, bias_r, gate_r, rows, causal, scale, offset)
+            o, lse = real(qr, k, v, bias_r, gate_r, rows, causal, scale, offset, mods)
             return o, lse / math.log(2.0)
         if kind == "gate_not_sigmoid" and gate_r is not None:
-            o, lse = real(qr, k, v, bias_r, None, rows, causal, scale, offset)
+            o, lse = real(qr, k, v, bias_r, None, rows, causal, scale, offset, mods)
             return o * gate_r, lse
         if kind == "transposed_q":
             qr = qr[::-1]
         if kind == "top_left_alignment":
             offset = 0
-        return real(qr, k, v, bias_r, gate_r, rows, causal, scale, offset)
+        return real(qr, k, v, bias_r, gate_r, rows, causal, scale, offset, mods)
 
     return attend
 
