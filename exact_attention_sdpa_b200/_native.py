@@ -22,13 +22,17 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIM
 ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
             "attn_debug_inject_stall", "attn_version")
 
 
 class AttnTensor(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int), ("ndim", ctypes.c_int32),
                 ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class AttnMods(ctypes.Structure):
+    _fields_ = [("alibi_slopes", ctypes.c_void_p), ("softcap", ctypes.c_float), ("window_left", ctypes.c_int32)]
 
 
 class AttnError(RuntimeError):
@@ -55,6 +59,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         P = ctypes.POINTER(AttnTensor)
         lib.attn_fwd.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd.restype = ctypes.c_int
+        lib.attn_fwd_ex.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, ctypes.POINTER(AttnMods), P,
+                                    ctypes.c_void_p, ctypes.c_void_p]
+        lib.attn_fwd_ex.restype = ctypes.c_int
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p,
                                       P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_host.restype = ctypes.c_int
@@ -108,25 +115,34 @@ def _ref(view: Optional[AttnTensor]):
     return None if view is None else ctypes.byref(view)
 
 
-def attn_fwd_raw(q, k, v, bias, gate, causal: bool, scale: float, out, lse, stream: int) -> int:
+def attn_fwd_raw(q, k, v, bias, gate, causal: bool, scale: float, out, lse, stream: int,
+                 softcap: float = 0.0, alibi_slopes: Optional[torch.Tensor] = None, window_left: int = -1) -> int:
     """Direct call of the C entry point with torch tensors; returns the status code."""
     lib = load_library()
     vq, vk, vv, vb, vg, vo = (make_view(t) for t in (q, k, v, bias, gate, out))
     lse_ptr = None if lse is None else lse.data_ptr()
-    return lib.attn_fwd(_ref(vq), _ref(vk), _ref(vv), _ref(vb), _ref(vg), int(bool(causal)), float(scale),
-                        _ref(vo), lse_ptr, stream)
+    if not softcap and alibi_slopes is None and window_left < 0:
+        return lib.attn_fwd(_ref(vq), _ref(vk), _ref(vv), _ref(vb), _ref(vg), int(bool(causal)), float(scale),
+                            _ref(vo), lse_ptr, stream)
+    mods = AttnMods(None if alibi_slopes is None else alibi_slopes.data_ptr(), float(softcap), int(window_left))
+    return lib.attn_fwd_ex(_ref(vq), _ref(vk), _ref(vv), _ref(vb), _ref(vg), int(bool(causal)), float(scale),
+                           ctypes.byref(mods), _ref(vo), lse_ptr, stream)
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[torch.Tensor] = None,
              gate: Optional[torch.Tensor] = None, causal: bool = False, scale: Optional[float] = None,
              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+             stream: Optional[torch.cuda.Stream] = None, softcap: float = 0.0,
+             alibi_slopes: Optional[torch.Tensor] = None, window_left: int = -1
+             ) -> Tuple[torch.Tensor, torch.Tensor]:
     """O = softmax(scale * Q K^T [+ bias]) V [* sigmoid(gate)] and the per-row logsumexp.
 
     q, k, v: CUDA tensors [B, H, N, d] (fp16 or bf16, d in {32, 64, 128}, last
     dim contiguous).  bias: [H, N, N] or [B, H, N, N]; gate: like q.  ``scale``
     defaults to 1/sqrt(d).  ``out``/``lse`` may be given preallocated.  The
     launch goes on ``stream`` (default: the current stream) and is asynchronous.
+    Optional score modifications (include/attn.h, attn_mods_t): ``alibi_slopes``
+    (CUDA fp32 [H]), ``softcap`` (> 0), ``window_left`` (>= 0).
     """
     if not q.is_cuda:
         raise ValueError("attn_fwd takes CUDA tensors; use fwd() for host tensors")
@@ -137,7 +153,7 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[t
     if lse is None:
         lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
-    _check(attn_fwd_raw(q, k, v, bias, gate, causal, scale, out, lse, s))
+    _check(attn_fwd_raw(q, k, v, bias, gate, causal, scale, out, lse, s, softcap, alibi_slopes, window_left))
     return out, lse
 
 

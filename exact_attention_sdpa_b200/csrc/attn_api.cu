@@ -169,9 +169,9 @@ struct Maps {
     CUtensorMap q, k, v, bias;
 };
 
-template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE>
+template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE, bool MODS = false>
 cudaError_t launch_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
-    auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE>;
+    auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE, MODS>;
     // At least 116 KB of dynamic shared memory, so that two CTAs (of two kernels running
     // concurrently on different streams) never share an SM: each CTA allocates all 512
     // tensor-memory columns, and a second one would only wait for the first to finish.
@@ -189,6 +189,11 @@ cudaError_t launch_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
 
 template <typename T, int D>
 cudaError_t launch_d(bool causal, bool bias, bool gate, const Maps& m, const FwdParams& p, cudaStream_t s) {
+    if (p.has_mods) {   // score modifications: built without bias and gate only
+        if (bias || gate) return cudaErrorInvalidValue;
+        return causal ? launch_t<T, D, true, false, false, true>(m, p, s)
+                      : launch_t<T, D, false, false, false, true>(m, p, s);
+    }
 #define ATTN_CASE(C, B_, G_) \
     if (causal == C && bias == B_ && gate == G_) return launch_t<T, D, C, B_, G_>(m, p, s);
     ATTN_CASE(false, false, false)
@@ -328,9 +333,22 @@ extern "C" {
 attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                        const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
                        attn_tensor_t* out, float* lse, cudaStream_t stream) {
+    return attn_fwd_ex(q, k, v, bias, gate, causal, scale, nullptr, out, lse, stream);
+}
+
+attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                          const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                          const attn_mods_t* mods, attn_tensor_t* out, float* lse, cudaStream_t stream) {
     bool empty = false;
     const attn_status_t st = validate_fwd(q, k, v, bias, gate, scale, out, lse, &empty);
-    if (st != ATTN_OK || empty) return st;
+    if (st != ATTN_OK) return st;
+    if (mods != nullptr) {
+        if (!std::isfinite(mods->softcap) || mods->softcap < 0.f) return ATTN_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(mods->alibi_slopes) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+        const bool on = mods->alibi_slopes != nullptr || mods->softcap > 0.f || mods->window_left >= 0;
+        if (on && (bias != nullptr || gate != nullptr)) return ATTN_ERR_UNSUPPORTED;
+    }
+    if (empty) return ATTN_OK;
     const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
 
     // ---- launch
@@ -389,6 +407,14 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     p.out_sh = out->stride[1];
     p.out_si = out->stride[2];
     p.lse = lse;
+    if (mods != nullptr) {
+        p.alibi = mods->alibi_slopes;
+        p.softcap = mods->softcap;
+        p.window_left = mods->window_left >= 0 ? mods->window_left : -1;
+        p.has_mods = (p.alibi != nullptr || p.softcap > 0.f || p.window_left >= 0) ? 1 : 0;
+    } else {
+        p.window_left = -1;
+    }
     p.wait_limit = g_wait_limit;
     p.status = status;
     p.inject_stall = g_inject_stall;

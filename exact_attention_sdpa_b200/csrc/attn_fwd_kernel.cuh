@@ -81,6 +81,11 @@ struct FwdParams {
     void* out;
     int64_t out_sb, out_sh, out_si;
     float* lse;                // nullable, [B*H*N]
+    // score modifications (generic path only), applied after scale and bias in this order:
+    const float* alibi;        // nullable [H]: s -= slope_h * |i + causal_off - j|
+    float softcap;             // > 0: s <- softcap * tanh(s / softcap)
+    int window_left;           // >= 0: keys j < i + causal_off - window_left are masked
+    int has_mods;              // any of the three is on
     unsigned long long wait_limit;
     unsigned int* status;
     int inject_stall;          // test hook: the MMA warp first waits on a barrier nothing arrives on
@@ -281,7 +286,8 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
     return U;
 }
 
-template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE>
+// MODS: score modifications compiled in (only without bias and gate); other builds carry none of it.
+template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE, bool MODS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
@@ -622,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t col_s = i ? Cfg<D>::kColS1 : Cfg<D>::kColS0;
         const uint32_t col_p = i ? Cfg<D>::kColP1 : Cfg<D>::kColP0;
         const float scale_log2 = p.scale_log2;
-        const bool fast = !HAS_BIAS && scale_log2 > 0.f;   // max over raw scores, fused scale
+        const bool fast = !HAS_BIAS && !MODS && scale_log2 > 0.f;   // max over raw scores, fused scale
         uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
         bool ok = true;
         for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
@@ -720,10 +726,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(&sh.bias_empty[i][bst]);
                         ++bcnt;
                     }
-                    if (need_mask) {
+                    int lo = 0;                        // first visible key of the tile (left window)
+                    if constexpr (MODS) {
+                        if (p.alibi != nullptr) {      // linear distance penalty of this head
+                            const float slope = p.alibi[U.h];
+                            const int dist0 = row + p.causal_off - kv0;
+#pragma unroll
+                            for (int c = 0; c < kBlockN; ++c)
+                                s[c] = fmaf(-slope, fabsf(static_cast<float>(dist0 - c)), s[c]);
+                        }
+                        if (p.softcap > 0.f) {         // c tanh(s / c), tanh(x) = 1 - 2 / (1 + e^2x)
+                            const float cap = p.softcap, k2 = 2.f * kLog2e / p.softcap;
+#pragma unroll
+                            for (int c = 0; c < kBlockN; ++c)
+                                s[c] = cap * (1.f - __fdividef(2.f, 1.f + ex2_approx(s[c] * k2)));
+                        }
+                        if (p.window_left >= 0) lo = row + p.causal_off - p.window_left - kv0;
+                    }
+                    if (need_mask || (MODS && p.window_left >= 0)) {
                         const int lim = CAUSAL ? min(p.Nk - kv0, row + p.causal_off - kv0 + 1) : (p.Nk - kv0);
 #pragma unroll
-                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim && c >= lo) ? s[c] : -INFINITY;
                     }
                     m_tile = row_max(s) * kLog2e;
                 }

@@ -102,6 +102,33 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
                        cudaStream_t stream);
 
 /*
+ * Optional score modifications (attention variants the pages list), applied
+ * after scale and bias, in this order, to the score s of query i and key j:
+ *   alibi_slopes  nullable; device fp32 [H]: s -= slope_h * |i + (Nk - N) - j|
+ *   softcap       > 0: s <- softcap * tanh(s / softcap); 0 turns it off
+ *   window_left   >= 0: keys j < i + (Nk - N) - window_left are masked (a left
+ *                 sliding window; with causal masking a band of window_left + 1
+ *                 keys); negative turns it off
+ * Key tiles left of every row's window are still visited (masked, not skipped).
+ */
+typedef struct {
+    const float* alibi_slopes;
+    float softcap;
+    int32_t window_left;
+} attn_mods_t;
+
+/*
+ * attn_fwd_ex -- attn_fwd with score modifications (`mods` nullable: none).
+ * Errors as attn_fwd, plus ATTN_ERR_INVALID_ARG for a negative or non-finite
+ * softcap or a misaligned alibi_slopes, and ATTN_ERR_UNSUPPORTED for a
+ * modification together with a bias or a gate.  attn_fwd(...) is
+ * attn_fwd_ex(..., NULL, ...).
+ */
+attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                          const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                          const attn_mods_t* mods, attn_tensor_t* out, float* lse, cudaStream_t stream);
+
+/*
  * attn_fwd_host -- the same operation end to end from HOST memory.
  *
  *   q, k, v, bias?, gate?   views of the inputs in host memory (layout rules of

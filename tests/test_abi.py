@@ -278,3 +278,17 @@ def test_backward_argument_checks(lib):
     e = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
     assert nat.attn_bwd_raw(e, k, v, e.clone(), None, e.clone(), False, 0.1, e.clone(), torch.zeros_like(k),
                             torch.zeros_like(v), 0) == nat.ATTN_OK                 # no query rows: nothing to do
+
+
+def test_modification_argument_checks(lib):
+    q, k, v, o = _qkv()
+    r = nat.attn_fwd_raw(q, k, v, None, None, False, 0.1, o, None, 0, softcap=-1.0)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+    r = nat.attn_fwd_raw(q, k, v, None, None, False, 0.1, o, None, 0, softcap=float("inf"))
+    assert r == nat.ATTN_ERR_INVALID_ARG
+    bias = torch.zeros(2, 64, 64, dtype=torch.float16)
+    r = nat.attn_fwd_raw(q, k, v, bias, None, False, 0.1, o, None, 0, window_left=4)
+    assert r == nat.ATTN_ERR_UNSUPPORTED                                       # modifications with a bias
+    bad = torch.zeros(3, dtype=torch.uint8)[1:]
+    r = nat.attn_fwd_raw(q, k, v, None, None, False, 0.1, o, None, 0, alibi_slopes=bad)
+    assert r == nat.ATTN_ERR_INVALID_ARG                                       # misaligned slopes
