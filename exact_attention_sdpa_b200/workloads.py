@@ -23,7 +23,7 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_grad_output", "attention_flops", "algorithmic_bytes"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_grad_output", "alibi_slopes", "attention_flops", "algorithmic_bytes"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -41,6 +41,9 @@ class Workload:
     gate: bool = False  # O <- sigmoid(G) * O, G has O's shape
     description: str = ""
     Nk: Optional[int] = None   # key rows when they differ from the N query rows (KV-cache shapes)
+    softcap: float = 0.0       # score modifications (0 / False / -1: off)
+    alibi: bool = False        # per-head slopes 2^(-8 (h+1) / H), see alibi_slopes()
+    window_left: int = -1
 
     @property
     def n_keys(self) -> int:
@@ -74,6 +77,10 @@ WORKLOADS: Dict[str, Workload] = {
                  bias=True, gate=True,
                  description="Evoformer-style gated row attention, R=256 H=8 N=256 d=32 bf16, "
                              "pair bias [H,N,N], sigmoid gate"),
+        Workload("n8192_alibi_softcap", B=4, H=12, N=8192, d=64, dtype="fp16", causal=True, seed=6,
+                 softcap=30.0, alibi=True,
+                 description="the B=4 H=12 N=8192 d=64 fp16 causal sizing with ALiBi slopes and a logit "
+                             "softcap of 30"),
         Workload("prefill_chunk", B=8, H=12, N=2048, d=64, dtype="fp16", causal=True, seed=5, Nk=8192,
                  description="a 2048-row prefill chunk against an 8192-row KV cache, B=8 H=12 d=64 fp16, "
                              "causal (bottom-right aligned)"),
@@ -143,3 +150,10 @@ def make_grad_output(w: Workload, seed: Optional[int] = None) -> torch.Tensor:
     g = torch.Generator(device="cpu")
     g.manual_seed((w.seed if seed is None else seed) + 1000)
     return torch.randn(w.B, w.H, w.N, w.d, generator=g, dtype=torch.float32).to(w.torch_dtype)
+
+
+def alibi_slopes(w: Workload) -> Optional[torch.Tensor]:
+    """The workload's ALiBi slopes (fp32 [H], the usual geometric 2^(-8 (h+1) / H)), or None."""
+    if not w.alibi:
+        return None
+    return torch.tensor([2.0 ** (-8.0 * (h + 1) / w.H) for h in range(w.H)], dtype=torch.float32)
