@@ -47,7 +47,7 @@ from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
-__all__ = ["sdpa_forward", "sdpa_rows", "sdpa_backward", "to_f64"]
+__all__ = ["sdpa_forward", "sdpa_rows", "sdpa_backward", "sdpa_varlen_forward", "to_f64"]
 
 
 def to_f64(x) -> Optional[np.ndarray]:
@@ -251,3 +251,37 @@ def sdpa_backward(q, k, v, do, causal: bool = False, scale: Optional[float] = No
             dQ[b, h], dK[b, h], dV[b, h] = _grad_rows(q[b, h], k[b, h], v[b, h], do[b, h], causal, scale,
                                                       k.shape[2] - Nq)
     return dQ, dK, dV
+
+
+# ---------------------------------------------------------------------------
+# ragged batches
+# ---------------------------------------------------------------------------
+
+def sdpa_varlen_forward(q, k, v, cu_q: Sequence[int], cu_k: Sequence[int], causal: bool = False,
+                        scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Sequences of different lengths packed along the token axis.
+
+    q: [Tq, H, d] with sequence b in rows cu_q[b] .. cu_q[b+1]; k, v: [Tk, H, d]
+    likewise with cu_k.  Each sequence is its own attention problem (no token
+    attends across a sequence boundary), with the bottom-right causal alignment
+    of sdpa_forward when its query and key counts differ.  Returns O [Tq, H, d]
+    and lse [H, Tq] in float64; a sequence with no query rows contributes nothing,
+    one with queries but no keys has dead rows (O = 0, lse = -inf).
+    """
+    q, k, v = (to_f64(t) for t in (q, k, v))
+    Tq, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    O = np.zeros((Tq, H, d))
+    L = np.full((H, Tq), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue
+        qs = q[q0:q1].transpose(1, 0, 2)[None]        # [1, H, n, d]
+        ks = k[k0:k1].transpose(1, 0, 2)[None]
+        vs = v[k0:k1].transpose(1, 0, 2)[None]
+        o, lse = sdpa_forward(qs, ks, vs, causal=causal, scale=scale)
+        O[q0:q1] = o[0].transpose(1, 0, 2)
+        L[:, q0:q1] = lse[0]
+    return O, L
