@@ -160,7 +160,16 @@ def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
     import numpy as np
 
     from oracle import sdpa_rows
-    inp = make_inputs(w)
+    if w.lengths is not None:                          # ragged: the longest sequence as one problem
+        from exact_attention_sdpa_b200.workloads import make_varlen_inputs
+        vi = make_varlen_inputs(w)
+        b0 = int(np.argmax(w.lengths))
+        r0, n = int(vi["cu_seqlens"][b0]), w.lengths[b0]
+        inp = {x: vi[x][r0:r0 + n].transpose(0, 1).unsqueeze(0) for x in "qkv"}
+        inp.update(bias=None, gate=None)
+        w = w.with_(B=1, N=n, lengths=None)
+    else:
+        inp = make_inputs(w)
     q, k, v = inp["q"], inp["k"], inp["v"]
     rng = np.random.default_rng(0)
     flops, secs = 0.0, 0.0
@@ -274,6 +283,64 @@ def run_bwd(args, w, config):
     print(json.dumps(line), flush=True)
 
 
+def run_varlen(args, w, config):
+    """A ragged batch on one GPU: K timed attn_fwd_varlen calls (one kernel launch per
+    sequence) after W warm-ups, packed inputs resident; the oracle times one sequence."""
+    from exact_attention_sdpa_b200 import attn_fwd_varlen, load_library
+    from exact_attention_sdpa_b200.workloads import make_varlen_inputs
+    load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_varlen_inputs(w)
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    cu = inp["cu_seqlens"]
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[1], q.shape[0], device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        attn_fwd_varlen(q, k, v, cu, cu, causal=w.causal, scale=w.scale, out=out, lse=lse, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    flops = attention_flops(w)
+    value = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"]
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded N(0,1) packed inputs)", "config": dict(config, lengths=list(w.lengths)),
+            "pct_of_peak": 100.0 * value / peak,
+            "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": None,
+                         "kernel": "attn_fwd_kernel (one launch per sequence)", "algorithmic_flops_per_launch": flops},
+            "gpu_launches": args.steps * sum(1 for n in w.lengths if n > 0), "e2e": None, "clocks": clocks.summary()}
+    if not args.no_cpu_baseline:
+        import numpy as np
+        from oracle import sdpa_rows
+        b = int(np.argmax(w.lengths))                 # the longest sequence, its last 1024 rows
+        r0, n = int(cu[b]), w.lengths[b]
+        qs, ks, vs = (inp[x][r0:r0 + n].transpose(0, 1).unsqueeze(0) for x in "qkv")
+        picks = [(0, h, i) for h in range(1) for i in range(max(0, n - 1024), n)]
+        t = time.perf_counter()
+        sdpa_rows(qs, ks, vs, picks, causal=w.causal, scale=w.scale)
+        dt = time.perf_counter() - t
+        vis = sum(i + 1 for (_, _, i) in picks)
+        line["cpu_baseline"] = {"value": 4.0 * w.d * vis / dt / 1e12, "unit": UNIT,
+                                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                                "sample": f"the last 1024 query rows of one head of the longest sequence ({n} tokens)"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -313,6 +380,8 @@ def main():
 
     if args.bwd:
         return run_bwd(args, w, config)
+    if w.lengths is not None:
+        return run_varlen(args, w, config)
     world, rank, local = dist_setup(args.gpus)
     from exact_attention_sdpa_b200 import attn_fwd, load_library
     load_library()

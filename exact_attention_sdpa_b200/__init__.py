@@ -8,8 +8,8 @@ The computation runs in ``libattn.so`` (built in-tree by
 arguments.  Importing it does not load the library; the first call does, and
 raises if the library is missing.
 """
-from ._native import (AttnError, Staging, attn_bwd, attn_fwd, attn_fwd_raw, fwd, last_device_status, load_library,
+from ._native import (AttnError, Staging, attn_bwd, attn_fwd, attn_fwd_raw, attn_fwd_varlen, fwd, last_device_status, load_library,
                       set_wait_limit, status_string, version)
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_fwd_raw", "fwd", "Staging", "AttnError", "last_device_status", "load_library",
+__all__ = ["attn_fwd", "attn_bwd", "attn_fwd_varlen", "attn_fwd_raw", "fwd", "Staging", "AttnError", "last_device_status", "load_library",
            "set_wait_limit", "status_string", "version"]

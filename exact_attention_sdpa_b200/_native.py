@@ -22,7 +22,7 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIM
 ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
             "attn_debug_inject_stall", "attn_version")
 
 
@@ -62,6 +62,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_fwd_ex.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, ctypes.POINTER(AttnMods), P,
                                     ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_ex.restype = ctypes.c_int
+        lib.attn_fwd_varlen.argtypes = [P, P, P, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int,
+                                        ctypes.c_float, P, ctypes.c_void_p, ctypes.c_void_p]
+        lib.attn_fwd_varlen.restype = ctypes.c_int
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p,
                                       P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_host.restype = ctypes.c_int
@@ -154,6 +157,36 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[t
         lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
     _check(attn_fwd_raw(q, k, v, bias, gate, causal, scale, out, lse, s, softcap, alibi_slopes, window_left))
+    return out, lse
+
+
+def attn_fwd_varlen_raw(q, k, v, cu_q, cu_k, causal: bool, scale: float, out, lse, stream: int) -> int:
+    """Direct call of attn_fwd_varlen; cu_q, cu_k are host int32 tensors of batch + 1 offsets."""
+    lib = load_library()
+    vq, vk, vv, vo = (make_view(t) for t in (q, k, v, out))
+    return lib.attn_fwd_varlen(_ref(vq), _ref(vk), _ref(vv), cu_q.data_ptr(), cu_k.data_ptr(), int(cu_q.numel() - 1),
+                               int(bool(causal)), float(scale), _ref(vo), None if lse is None else lse.data_ptr(), stream)
+
+
+def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q, cu_seqlens_k,
+                    causal: bool = False, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Ragged batch packed along the token axis: q [Tq, H, d], k, v [Tk, H, d] (CUDA);
+    sequence b owns rows cu_seqlens_q[b]..cu_seqlens_q[b+1] of q (cu_seqlens_k for k, v).
+    The offsets are read on the host.  Returns O [Tq, H, d] and lse [H, Tq]."""
+    if not q.is_cuda:
+        raise ValueError("attn_fwd_varlen takes CUDA tensors")
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    cu_q = torch.as_tensor(cu_seqlens_q, dtype=torch.int32).cpu().contiguous()
+    cu_k = torch.as_tensor(cu_seqlens_k, dtype=torch.int32).cpu().contiguous()
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty(q.shape[1], q.shape[0], device=q.device, dtype=torch.float32)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(attn_fwd_varlen_raw(q, k, v, cu_q, cu_k, causal, scale, out, lse, s))
     return out, lse
 
 

@@ -326,6 +326,12 @@ bool same_layout(const attn_tensor_t* a, const attn_tensor_t* b) {
     return true;
 }
 
+// attn_fwd_ex with an optional lse layout (defined below the C entry points)
+attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                       const attn_mods_t* mods, attn_tensor_t* out, float* lse, const int64_t* lse_layout,
+                       cudaStream_t stream);
+
 }  // namespace
 
 extern "C" {
@@ -339,6 +345,17 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
 attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                           const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
                           const attn_mods_t* mods, attn_tensor_t* out, float* lse, cudaStream_t stream) {
+    return fwd_impl(q, k, v, bias, gate, causal, scale, mods, out, lse, nullptr, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// attn_fwd_ex with an optional lse layout {stride between batches, stride between heads}
+attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                       const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                       const attn_mods_t* mods, attn_tensor_t* out, float* lse, const int64_t* lse_layout,
+                       cudaStream_t stream) {
     bool empty = false;
     const attn_status_t st = validate_fwd(q, k, v, bias, gate, scale, out, lse, &empty);
     if (st != ATTN_OK) return st;
@@ -407,6 +424,12 @@ attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const 
     p.out_sh = out->stride[1];
     p.out_si = out->stride[2];
     p.lse = lse;
+    p.lse_sh = N;
+    p.lse_sb = H * N;
+    if (lse_layout != nullptr) {   // (ragged batches: each sequence's rows inside [H, T])
+        p.lse_sb = lse_layout[0];
+        p.lse_sh = lse_layout[1];
+    }
     if (mods != nullptr) {
         p.alibi = mods->alibi_slopes;
         p.softcap = mods->softcap;
@@ -428,6 +451,10 @@ attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const 
                                  stream);
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
+
+}  // namespace
+
+extern "C" {
 
 attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                             const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
@@ -467,6 +494,58 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
     if (lse != nullptr) {
         const size_t n = static_cast<size_t>(q->shape[0] * q->shape[1] * q->shape[2]) * sizeof(float);
         if (cudaMemcpyAsync(lse, lse_dev, n, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
+attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch, int causal,
+                              float scale, attn_tensor_t* out, float* lse, cudaStream_t stream) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (q->dtype == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+    if (!is_half_type(q->dtype)) return ATTN_ERR_INVALID_ARG;
+    if (k->dtype != q->dtype || v->dtype != q->dtype || out->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
+    if (q->ndim != 3 || k->ndim != 3 || v->ndim != 3 || out->ndim != 3) return ATTN_ERR_INVALID_ARG;
+    if (!same_shape(k, v) || !same_shape(q, out)) return ATTN_ERR_INVALID_ARG;
+    if (q->shape[1] != k->shape[1] || q->shape[2] != k->shape[2]) return ATTN_ERR_INVALID_ARG;
+    if (batch < 0 || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    const int64_t Tq = q->shape[0], Tk = k->shape[0], H = q->shape[1];
+    if (cu_seqlens_q[0] != 0 || cu_seqlens_k[0] != 0 || cu_seqlens_q[batch] != Tq || cu_seqlens_k[batch] != Tk)
+        return ATTN_ERR_INVALID_ARG;
+    for (int32_t b = 0; b < batch; ++b) {
+        const int32_t nq = cu_seqlens_q[b + 1] - cu_seqlens_q[b], nk = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+        if (nq < 0 || nk < 0) return ATTN_ERR_INVALID_ARG;
+        if (nq > 0 && nk == 0) return ATTN_ERR_INVALID_ARG;     // queries with no key at all
+    }
+    if (Tq == 0 || H == 0) return ATTN_OK;
+    // each sequence: a [1, H, n, d] view of the packed [T, H, d] tensors (strides in elements);
+    // every check of attn_fwd runs on the first sequence's views before anything is launched
+    auto view = [](const attn_tensor_t* t, int64_t row0, int64_t n) {
+        attn_tensor_t x;
+        x.data = static_cast<char*>(t->data) + row0 * t->stride[0] * 2;
+        x.dtype = t->dtype;
+        x.ndim = 4;
+        x.shape[0] = 1; x.shape[1] = t->shape[1]; x.shape[2] = n; x.shape[3] = t->shape[2];
+        x.stride[0] = n * t->stride[0]; x.stride[1] = t->stride[1]; x.stride[2] = t->stride[0]; x.stride[3] = t->stride[2];
+        return x;
+    };
+    const int64_t lse_layout[2] = {0, Tq};
+    for (int pass = 0; pass < 2; ++pass) {        // pass 0: validate every sequence; pass 1: launch
+        for (int32_t b = 0; b < batch; ++b) {
+            const int64_t q0 = cu_seqlens_q[b], nq = cu_seqlens_q[b + 1] - q0;
+            const int64_t k0 = cu_seqlens_k[b], nk = cu_seqlens_k[b + 1] - k0;
+            if (nq == 0) continue;
+            attn_tensor_t vq = view(q, q0, nq), vk = view(k, k0, nk), vv = view(v, k0, nk), vo = view(out, q0, nq);
+            bool empty = false;
+            attn_status_t st = validate_fwd(&vq, &vk, &vv, nullptr, nullptr, scale, &vo, lse, &empty);
+            if (st != ATTN_OK) return st;
+            if (pass == 1) {
+                st = fwd_impl(&vq, &vk, &vv, nullptr, nullptr, causal, scale, nullptr, &vo,
+                              lse == nullptr ? nullptr : lse + q0, lse_layout, stream);
+                if (st != ATTN_OK) return st;
+            }
+        }
     }
     return ATTN_OK;
 }

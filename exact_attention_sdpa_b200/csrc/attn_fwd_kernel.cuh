@@ -80,7 +80,8 @@ struct FwdParams {
     int64_t gate_sb, gate_sh, gate_si;
     void* out;
     int64_t out_sb, out_sh, out_si;
-    float* lse;                // nullable, [B*H*N]
+    float* lse;                // nullable; row (b, h, i) at b * lse_sb + h * lse_sh + i
+    int64_t lse_sb, lse_sh;
     // score modifications (generic path only), applied after scale and bias in this order:
     const float* alibi;        // nullable [H]: s -= slope_h * |i + causal_off - j|
     float softcap;             // > 0: s <- softcap * tanh(s / softcap)
@@ -945,7 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     finish_chunk(r, c);
                 }
                 if (p.lse != nullptr && row_ok)
-                    p.lse[static_cast<int64_t>(U.bh) * p.N + row] =
+                    p.lse[U.b * p.lse_sb + U.h * p.lse_sh + row] =
                         (l > 0.f) ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
             }
         }

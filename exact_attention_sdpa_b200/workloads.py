@@ -23,7 +23,7 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_grad_output", "alibi_slopes", "attention_flops", "algorithmic_bytes"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_grad_output", "make_varlen_inputs", "alibi_slopes", "attention_flops", "algorithmic_bytes"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -44,6 +44,7 @@ class Workload:
     softcap: float = 0.0       # score modifications (0 / False / -1: off)
     alibi: bool = False        # per-head slopes 2^(-8 (h+1) / H), see alibi_slopes()
     window_left: int = -1
+    lengths: Optional[tuple] = None   # ragged batch: per-sequence token counts (B = len, N = max)
 
     @property
     def n_keys(self) -> int:
@@ -81,6 +82,10 @@ WORKLOADS: Dict[str, Workload] = {
                  softcap=30.0, alibi=True,
                  description="the B=4 H=12 N=8192 d=64 fp16 causal sizing with ALiBi slopes and a logit "
                              "softcap of 30"),
+        Workload("varlen_mix", B=16, H=12, N=4096, d=64, dtype="fp16", causal=True, seed=7,
+                 lengths=(3072, 512, 1911, 4096, 256, 2600, 1024, 3333, 768, 1500, 4000, 2048, 300, 2900, 1200, 3600),
+                 description="a ragged batch of 16 sequences of 256-4096 tokens (36,920 in all), H=12 d=64 "
+                             "fp16, causal, packed along the token axis"),
         Workload("prefill_chunk", B=8, H=12, N=2048, d=64, dtype="fp16", causal=True, seed=5, Nk=8192,
                  description="a 2048-row prefill chunk against an 8192-row KV cache, B=8 H=12 d=64 fp16, "
                              "causal (bottom-right aligned)"),
@@ -115,10 +120,33 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional[t
     return {"q": q, "k": k, "v": v, "bias": bias, "gate": gate}
 
 
+def make_varlen_inputs(w: Workload, seed: Optional[int] = None):
+    """Packed inputs of a ragged workload: q, k, v [T, H, d] (T = sum of lengths) drawn as
+    make_inputs does, and the host int32 offsets cu_seqlens (batch + 1 entries)."""
+    assert w.lengths is not None
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    T = sum(w.lengths)
+
+    def draw():
+        x = torch.randn(T, w.H, w.d, generator=g, dtype=torch.float32)
+        if w.amp != 1.0:
+            x.mul_(w.amp)
+        return x.to(w.torch_dtype)
+
+    q, k, v = draw(), draw(), draw()
+    cu = torch.zeros(len(w.lengths) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(w.lengths, dtype=torch.int64), 0).to(torch.int32)
+    return {"q": q, "k": k, "v": v, "cu_seqlens": cu}
+
+
 def attention_flops(w: Workload) -> float:
     """The metric's FLOP count: 4*B*H*N^2*d, halved for causal (square problems).  With
     Nk keys: 4*B*H*d times the number of visible (query, key) pairs, N*Nk without causal
     masking, and with it the pairs j <= i + (Nk - N) (N*Nk - N*(N-1)/2 when N <= Nk)."""
+    if w.lengths is not None:
+        f = sum(4.0 * w.H * n * n * w.d for n in w.lengths)
+        return f / 2.0 if w.causal else f
     if w.Nk is None:
         f = 4.0 * w.B * w.H * w.N * w.N * w.d
         return f / 2.0 if w.causal else f
@@ -134,6 +162,9 @@ def attention_flops(w: Workload) -> float:
 def algorithmic_bytes(w: Workload) -> int:
     """Bytes one forward must move at least once: Q, K, V (and G, bias) read, O and lse written."""
     elem = 2
+    if w.lengths is not None:                     # q, k, v, o of every token, lse
+        T = sum(w.lengths)
+        return 4 * T * w.H * w.d * elem + T * w.H * 4
     per_q = w.B * w.H * w.N * w.d * elem
     per_kv = w.B * w.H * w.n_keys * w.d * elem
     per_tensor = per_q

@@ -129,6 +129,30 @@ attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const 
                           const attn_mods_t* mods, attn_tensor_t* out, float* lse, cudaStream_t stream);
 
 /*
+ * attn_fwd_varlen -- a batch of sequences of different lengths, packed along
+ * the token axis (each sequence is its own attention problem; no token attends
+ * across a sequence boundary).
+ *
+ *   q, out     [Tq, H, d] device views; sequence b owns rows
+ *              cu_seqlens_q[b] .. cu_seqlens_q[b+1]
+ *   k, v       [Tk, H, d]; sequence b owns rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]
+ *   cu_seqlens_q, cu_seqlens_k
+ *              HOST int32 arrays of batch + 1 non-decreasing offsets, starting
+ *              at 0 and ending at Tq (resp. Tk)
+ *   causal     per sequence, aligned at the bottom right as in attn_fwd
+ *   lse        nullable; [H, Tq] fp32, row (h, t) at h * Tq + t
+ *
+ * Layout rules as attn_fwd (unit inner stride, other strides multiples of 16
+ * bytes, 16-byte aligned data).  A sequence with no query rows is skipped; one
+ * with query rows but no key rows is ATTN_ERR_INVALID_ARG.  Every sequence is
+ * checked before the first launch.  This version launches the fused kernel
+ * once per non-empty sequence, in order, on `stream`.
+ */
+attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch, int causal,
+                              float scale, attn_tensor_t* out, float* lse, cudaStream_t stream);
+
+/*
  * attn_fwd_host -- the same operation end to end from HOST memory.
  *
  *   q, k, v, bias?, gate?   views of the inputs in host memory (layout rules of

@@ -292,3 +292,24 @@ def test_modification_argument_checks(lib):
     bad = torch.zeros(3, dtype=torch.uint8)[1:]
     r = nat.attn_fwd_raw(q, k, v, None, None, False, 0.1, o, None, 0, alibi_slopes=bad)
     assert r == nat.ATTN_ERR_INVALID_ARG                                       # misaligned slopes
+
+
+def test_varlen_argument_checks(lib):
+    q = torch.zeros(10, 2, 64, dtype=torch.float16)
+    k = torch.zeros(12, 2, 64, dtype=torch.float16)
+    o = torch.zeros_like(q)
+    ok_q = torch.tensor([0, 4, 10], dtype=torch.int32)
+    ok_k = torch.tensor([0, 5, 12], dtype=torch.int32)
+
+    def call_v(cq, ck, q_=q, k_=k, o_=o):
+        return nat.attn_fwd_varlen_raw(q_, k_, k_.clone(), cq, ck, True, 0.1, o_, None, 0)
+
+    assert call_v(torch.tensor([0, 4, 9], dtype=torch.int32), ok_k) == nat.ATTN_ERR_INVALID_ARG   # does not end at Tq
+    assert call_v(torch.tensor([1, 4, 10], dtype=torch.int32), ok_k) == nat.ATTN_ERR_INVALID_ARG  # does not start at 0
+    assert call_v(torch.tensor([0, 11, 10], dtype=torch.int32), ok_k) == nat.ATTN_ERR_INVALID_ARG  # decreasing
+    assert call_v(ok_q, torch.tensor([0, 0, 12], dtype=torch.int32)) == nat.ATTN_ERR_INVALID_ARG   # queries, no keys
+    assert call_v(ok_q, ok_k, q_=q.unsqueeze(0)) == nat.ATTN_ERR_INVALID_ARG                       # rank 4
+    assert call_v(ok_q, ok_k, k_=torch.zeros(12, 2, 32, dtype=torch.float16)) == nat.ATTN_ERR_INVALID_ARG
+    e = torch.zeros(0, 2, 64, dtype=torch.float16)
+    z = torch.zeros(1, dtype=torch.int32)
+    assert nat.attn_fwd_varlen_raw(e, e, e.clone(), z, z, True, 0.1, e.clone(), None, 0) == nat.ATTN_OK
