@@ -233,6 +233,15 @@ def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
             "api": "fwd() -> attn_fwd_host (C ABI, pinned host buffers), 2 streams"}
 
 
+def launch_percentiles(ms):
+    """p10 / median / p90 of per-launch device times (nearest-rank on the sorted list)."""
+    xs = sorted(ms)
+    if not xs:
+        return {"p10": None, "p50": None, "p90": None}
+    pick = lambda q: xs[min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))]
+    return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90)}
+
+
 def fp32_fma_peak_tflops(sm_mhz: float) -> float:
     """FP32 FMA peak of a B200: 148 SMs x 128 FP32 lanes x 2 FLOP per clock."""
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -465,6 +474,7 @@ def main():
                          "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "traffic": load_traffic(w.name), "kernel": "attn_fwd_kernel",
                          "mean_launch_ms": mean_launch_ms,
+                         "launch_ms_percentiles": launch_percentiles(launch_ms),
                          "algorithmic_flops_per_launch": flops},
             "gpu_launches": args.steps,
             "e2e": e2e,

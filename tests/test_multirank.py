@@ -61,3 +61,11 @@ def test_reference_arm_prints_from_rank_zero_only():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
                         "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_launch_percentiles():
+    sys.path.insert(0, ROOT)
+    import bench
+    p = bench.launch_percentiles([float(x) for x in range(1, 12)])   # 1..11
+    assert p == {"p10": 2.0, "p50": 6.0, "p90": 10.0}
+    assert bench.launch_percentiles([0.5]) == {"p10": 0.5, "p50": 0.5, "p90": 0.5}
