@@ -313,3 +313,42 @@ def test_varlen_argument_checks(lib):
     e = torch.zeros(0, 2, 64, dtype=torch.float16)
     z = torch.zeros(1, dtype=torch.int32)
     assert nat.attn_fwd_varlen_raw(e, e, e.clone(), z, z, True, 0.1, e.clone(), None, 0) == nat.ATTN_OK
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "attn.h"
+int main(void) {
+    /* host-side calls only: no device work */
+    if (strchr(attn_version(), '.') == NULL) return 1;
+    if (attn_status_string(ATTN_ERR_TIMEOUT) == NULL) return 2;
+    attn_tensor_t q;
+    memset(&q, 0, sizeof(q));
+    if (attn_fwd(NULL, &q, &q, NULL, NULL, 0, 0.125f, &q, NULL, 0) != ATTN_ERR_INVALID_ARG) return 3;
+    q.dtype = ATTN_F32;
+    if (attn_fwd(&q, &q, &q, NULL, NULL, 0, 0.125f, &q, NULL, 0) != ATTN_ERR_UNSUPPORTED) return 4;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_calls(lib, tmp_path):
+    """The boundary is a C ABI: a C99 program includes the header, links libattn.so and
+    gets the documented status codes (host-side checks only)."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(nat.LIB_PATH)
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                        str(src), "-L", libdir, "-lattn", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
