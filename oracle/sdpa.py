@@ -1,4 +1,6 @@
-"""fp64 CPU oracle for the exact scaled-dot-product attention forward.
+"""fp64 CPU oracle for the exact scaled-dot-product attention: the forward
+(sdpa_forward, sdpa_rows), ragged batches (sdpa_varlen_forward) and the
+gradients (sdpa_backward).
 
 TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
 and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may
@@ -39,7 +41,8 @@ exponentials shifted by it.  Readings of points the pages leave open:
   sliding window, together with the causal mask a band of w + 1 keys).
 
 Inputs of any float dtype are upcast exactly to float64 before any arithmetic.
-Parity: pinned (see tests/test_oracle.py for the pins).
+Parity: every function is pinned (tests/test_oracle.py, test_oracle_mods.py,
+test_oracle_varlen.py, test_oracle_backward.py, test_oracle_properties.py).
 """
 from __future__ import annotations
 
