@@ -69,3 +69,19 @@ def test_launch_percentiles():
     p = bench.launch_percentiles([float(x) for x in range(1, 12)])   # 1..11
     assert p == {"p10": 2.0, "p50": 6.0, "p90": 10.0}
     assert bench.launch_percentiles([0.5]) == {"p10": 0.5, "p50": 0.5, "p90": 0.5}
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    h = bench.kernel_source_hash()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "ncu_traffic.json").write_text(json.dumps({
+        "a": {"kernel_source_sha": h, "dram_bytes_per_launch": 123},
+        "b": {"kernel_source_sha": "0" * 16, "dram_bytes_per_launch": 456}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: h)
+    assert bench.load_traffic("a") == 123
+    assert bench.load_traffic("b") is None          # captured on another kernel source
+    assert bench.load_traffic("missing") is None
