@@ -1,9 +1,9 @@
 """ctypes binding of libattn.so (argument marshalling only).
 
-Every step of the attention forward runs in the library's CUDA kernel; this
-module converts torch tensors into the C ABI's ``attn_tensor_t`` views, passes
-the current CUDA stream and turns status codes into exceptions.  There is no
-fallback: if the shared library is missing the call raises.
+Every step of the attention forward and backward runs in the library's CUDA
+kernels; this module converts torch tensors into the C ABI's ``attn_tensor_t``
+views, passes the current CUDA stream and turns status codes into exceptions.
+There is no fallback: if the shared library is missing the call raises.
 """
 from __future__ import annotations
 
