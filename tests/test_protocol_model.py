@@ -1,0 +1,78 @@
+"""The forward kernel's mbarrier protocol, executed as a model under random schedules (CPU).
+
+tests/protocol_model.py restates the barrier protocol of attn_fwd_kernel.cuh (one actor per
+warp, asynchronous tensor-core and TMA work, version-tagged buffers).  These tests run it over
+the kernel's configurations (separate P columns at d <= 64 or P inside S at d = 128, causal or
+not, K/V ring depths 2-4, staged bias tiles) and over random unit sequences, including units of
+a single key tile and causal units whose second query tile reaches one more key tile than the
+first.  Every run must finish without a stale read, a parity-aliased wait or a deadlock.  The
+last test plants protocol mistakes of the kinds a change to the kernel could make and checks
+that the model finds each of them.
+"""
+import random
+
+import pytest
+
+import protocol_model as pm
+
+CONFIGS = [
+    # (separate_p, causal, stages, bias_stages): the kernel's instantiations at d = 32, 64, 128
+    (True, True, 4, 0), (True, True, 4, 2), (True, False, 4, 2),     # d = 32 (bias: 2 stages)
+    (True, True, 3, 0), (True, False, 3, 0), (True, True, 3, 1), (True, False, 3, 1),   # d = 64
+    (False, True, 2, 0), (False, False, 2, 0),                        # d = 128
+    (True, True, 2, 0), (False, True, 3, 0),                          # other ring depths
+]
+
+
+@pytest.mark.parametrize("sep,causal,stages,bias", CONFIGS)
+def test_protocol_holds_under_random_schedules(sep, causal, stages, bias):
+    for rep in range(40):
+        rng = random.Random(1000 * stages + 10 * bias + rep)
+        cfg = pm.Config(separate_p=sep, causal=causal, stages=stages, bias_stages=bias,
+                        units=pm.random_units(rng, causal, rng.randint(1, 4)))
+        pm.run(cfg, seed=rep)
+
+
+@pytest.mark.parametrize("sep", [True, False])
+def test_protocol_holds_over_long_unit_sequences(sep):
+    # many units per CTA: every parity counter wraps many times
+    for rep in range(6):
+        rng = random.Random(77 + rep)
+        cfg = pm.Config(separate_p=sep, causal=True, stages=3 if sep else 2,
+                        units=pm.random_units(rng, True, 12, max_tiles=3))
+        pm.run(cfg, seed=rep)
+
+
+def test_single_tile_units_back_to_back():
+    # units with one key tile each: S_i(0) of the next unit, Q release and the statistics
+    # double buffer are exercised on every unit
+    for rep in range(20):
+        cfg = pm.Config(separate_p=rep % 2 == 0, causal=True, stages=3,
+                        units=[(1, 1 + (rep + u) % 2) for u in range(6)])
+        pm.run(cfg, seed=rep)
+
+
+PLANTS = {
+    "empty_parity": True,           # producer waits the K/V release of the wrong phase
+    "no_s_free_wait": True,         # S_0(j+1) issued before the softmax read S_0(j)
+    "s_before_pv": False,           # d = 128: S_0(j+1) overwrites P_0(j) before PV_0(j)
+    "alpha_before_o_done": True,    # alpha(j) published before PV_i(j-1) completed
+    "no_o_done_wait": True,         # P_i(j) written while PV_i(j-1) may still read P_i(j-1)
+    "stats_no_o_free_wait": True,   # final m, l published before the previous epilogue read them
+    "arrive_before_rescale": True,  # correction releases PV_i(j) before rescaling O_i
+}
+
+
+@pytest.mark.parametrize("plant", sorted(PLANTS))
+def test_model_finds_planted_mistakes(plant):
+    sep = PLANTS[plant]
+    for rep in range(400):
+        rng = random.Random(rep)
+        causal = rep % 2 == 0
+        cfg = pm.Config(separate_p=sep, causal=causal, stages=2 + rep % 3,
+                        units=pm.random_units(rng, causal, rng.randint(1, 4)), plant=plant)
+        try:
+            pm.run(cfg, seed=rep)
+        except pm.ProtocolError:
+            return
+    pytest.fail(f"planted mistake {plant!r} went unnoticed in 400 schedules")
