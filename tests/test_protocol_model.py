@@ -76,3 +76,27 @@ def test_model_finds_planted_mistakes(plant):
         except pm.ProtocolError:
             return
     pytest.fail(f"planted mistake {plant!r} went unnoticed in 400 schedules")
+
+
+def test_model_barriers_match_the_kernel_source():
+    # The model must know every mbarrier the kernel initialises, with the same arrival count;
+    # a barrier added to or re-counted in the kernel without the model fails here.
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "exact_attention_sdpa_b200", "csrc",
+                            "attn_fwd_kernel.cuh")).read()
+    found = {}
+    for name, expr in re.findall(r"mbar_init\(&sh\.(\w+)(?:\[[^\]]*\])*,\s*([^;]+)\);", src):
+        found[name] = eval(expr.strip(), {"kBlockM": 128})
+    found.pop("never")            # stall-injection target: nothing ever arrives on it
+    st = pm.State(pm.Config(units=[(1, 1)], bias_stages=1))
+    model = {}
+    for name, val in vars(st).items():
+        bars = val
+        while isinstance(bars, list) and bars and isinstance(bars[0], list):
+            bars = bars[0]
+        if isinstance(bars, list) and bars and isinstance(bars[0], pm.Barrier):
+            model[name] = bars[0].count
+        elif isinstance(val, pm.Barrier):
+            model[name] = val.count
+    assert found == model
