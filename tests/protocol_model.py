@@ -18,8 +18,9 @@ in the kernel, one actor per warp, and executes it on the CPU under random sched
     exactly the version the kernel means to read.
 
 A run fails on a stale or early read (a race), on a wait that returns while its barrier is not
-exactly one phase past the phase the waiter means (parity aliasing), or on a state where no
-actor can move (deadlock).  The model is a restatement of the kernel's control flow, not the
+exactly one phase past the phase the waiter means (parity aliasing), on a state where no
+actor can move (deadlock), or, when a bounded wait was made to give up (Config.timeout), on a
+teardown reached while a TMA load or a tensor-core operation is still in flight.  The model is a restatement of the kernel's control flow, not the
 kernel itself: a change to the kernel's barrier protocol has to be mirrored here.
 """
 from __future__ import annotations
@@ -57,6 +58,7 @@ class Wait:
     bar: Barrier
     parity: int
     phase: int          # the phase the waiter means (its completion); parity must equal phase & 1
+    drain: bool = False  # a drain wait on exit: ignores the abort flag (the kernel's drain_phase)
 
 
 @dataclass
@@ -100,6 +102,7 @@ class Config:
     bias_stages: int = 0          # staged bias tiles per query tile (0: no bias through TMA)
     units: list = field(default_factory=list)    # per unit (nkv0, nkv1)
     plant: str = ""               # a protocol mistake planted on purpose (tests of the checker)
+    timeout: tuple = ()           # (role, n): that role's n-th bounded wait gives up (abort path)
 
 
 def random_units(rng: random.Random, causal: bool, n_units: int, max_tiles: int = 5) -> list:
@@ -134,6 +137,8 @@ class State:
         self.bias_full = [[B(f"bias_full{i}.{s}", 1) for s in range(BS)] for i in range(2)]
         self.bias_empty = [[B(f"bias_empty{i}.{s}", 128) for s in range(BS)] for i in range(2)]
         self.drain = B("drain", 1)
+        self.teardown = B("teardown", 14)             # __syncthreads before tensor memory is freed
+        self.abort = False                            # the CTA's abort flag
         # buffers (version tags)
         self.sQ = [None, None]
         self.sK = [None] * ST
@@ -152,40 +157,61 @@ class State:
 
 
 # ---------------------------------------------------------------------------------------- roles
+# Each role mirrors its branch of the kernel, including what it does when a bounded wait gives
+# up: `ok = yield Wait(...)` is False after a timeout or once another role raised the abort flag,
+# and the role then leaves its loops the way the kernel does, drains, and meets the others at
+# the teardown barrier.
+
 def nkv_of(cfg: Config, k: int, i: int) -> int:
     return cfg.units[k][i]
 
 
+def teardown(st: State):
+    yield Arrive(st.teardown, 1)
+    yield Wait(st.teardown, 0, 0, drain=True)
+
+
 def producer(st: State):
-    """TMA producer warp: Q0, K(0), Q1, V(0), [bias], then K(j), V(j), [bias] per unit."""
+    """TMA producer warp: Q0, K(0), Q1, V(0), [bias], then K(j), V(j), [bias] per unit; drains."""
     cfg, ST, BS = st.cfg, st.cfg.stages, st.cfg.bias_stages
-    kc = vc = 0
+    cnt = {"K": 0, "V": 0}
     qc = [0, 0]
     bc = [0, 0]
+    ok = True
+
+    def WU(bar, parity, phase):
+        nonlocal ok
+        if ok:
+            ok = yield Wait(bar, parity, phase)
+        return ok
 
     def load_q(i, k):
-        if qc[i] > 0:
-            yield Wait(st.q_empty[i], (qc[i] - 1) & 1, qc[i] - 1)
+        if qc[i] > 0 and not (yield from WU(st.q_empty[i], (qc[i] - 1) & 1, qc[i] - 1)):
+            return
 
         def run(s, i=i, k=k):
             s.sQ[i] = k
         yield Tma(f"Q{i} unit {k}", run, st.q_full[i])
         qc[i] += 1
 
-    def load_kv(kind, ring_full, ring_empty, buf, cnt, tile_id):
-        s_ = cnt % ST
-        if cnt >= ST:
-            par = (cnt // ST) & 1 if cfg.plant == "empty_parity" else ((cnt // ST) - 1) & 1
-            yield Wait(ring_empty[s_], par, cnt // ST - 1)
+    def load_kv(kind):
+        full, empty, buf = ((st.k_full, st.k_empty, "sK") if kind == "K" else (st.v_full, st.v_empty, "sV"))
+        n = cnt[kind]
+        s_ = n % ST
+        if n >= ST:
+            par = (n // ST) & 1 if cfg.plant == "empty_parity" else ((n // ST) - 1) & 1
+            if not (yield from WU(empty[s_], par, n // ST - 1)):
+                return
 
-        def run(s, s_=s_, tile_id=tile_id):
+        def run(s, s_=s_, tile_id=n):
             getattr(s, buf)[s_] = tile_id
-        yield Tma(f"{kind} tile {tile_id}", run, ring_full[s_])
+        yield Tma(f"{kind} tile {n}", run, full[s_])
+        cnt[kind] += 1
 
     def load_bias(i, j, k):
         s_ = bc[i] % BS
-        if bc[i] >= BS:
-            yield Wait(st.bias_empty[i][s_], ((bc[i] // BS) - 1) & 1, bc[i] // BS - 1)
+        if bc[i] >= BS and not (yield from WU(st.bias_empty[i][s_], ((bc[i] // BS) - 1) & 1, bc[i] // BS - 1)):
+            return
 
         def run(s, i=i, s_=s_, j=j, k=k):
             s.sBias[i][s_] = (k, j)
@@ -193,24 +219,49 @@ def producer(st: State):
         bc[i] += 1
 
     for k, (n0, n1) in enumerate(cfg.units):
+        if not ok:
+            break
         yield from load_q(0, k)
-        yield from load_kv("K", st.k_full, st.k_empty, "sK", kc, kc)
-        kc += 1
-        yield from load_q(1, k)
-        yield from load_kv("V", st.v_full, st.v_empty, "sV", vc, vc)
-        vc += 1
+        if ok:
+            yield from load_kv("K")
+        if ok:
+            yield from load_q(1, k)
+        if ok:
+            yield from load_kv("V")
         if BS:
-            yield from load_bias(0, 0, k)
-            yield from load_bias(1, 0, k)
-        for j in range(1, n1):
-            yield from load_kv("K", st.k_full, st.k_empty, "sK", kc, kc)
-            kc += 1
-            yield from load_kv("V", st.v_full, st.v_empty, "sV", vc, vc)
-            vc += 1
+            if ok:
+                yield from load_bias(0, 0, k)
+            if ok:
+                yield from load_bias(1, 0, k)
+        j = 1
+        while ok and j < n1:
+            yield from load_kv("K")
+            if ok:
+                yield from load_kv("V")
             if BS:
-                if j < n0:
+                if ok and j < n0:
                     yield from load_bias(0, j, k)
-                yield from load_bias(1, j, k)
+                if ok:
+                    yield from load_bias(1, j, k)
+            j += 1
+    # every load issued into shared memory lands before the CTA exits
+    if cfg.plant == "no_tma_drain":
+        yield from teardown(st)
+        return
+    for i in range(2):
+        if qc[i] > 0:
+            yield Wait(st.q_full[i], (qc[i] - 1) & 1, qc[i] - 1, drain=True)
+    for s_ in range(ST):
+        for kind, full in (("K", st.k_full), ("V", st.v_full)):
+            if cnt[kind] > s_:
+                n = (cnt[kind] - 1 - s_) // ST
+                yield Wait(full[s_], n & 1, n, drain=True)
+    for i in range(2):
+        for s_ in range(BS):
+            if bc[i] > s_:
+                n = (bc[i] - 1 - s_) // BS
+                yield Wait(st.bias_full[i][s_], n & 1, n, drain=True)
+    yield from teardown(st)
 
 
 def s_mma(st: State, i: int, k: int, j: int, kst: int, key_tile: int):
@@ -247,100 +298,126 @@ def mma_issuer(st: State):
     pv_cnt, sf_cnt = [0, 0], [0, 0]
     early = [False, False]
     n_units = len(cfg.units)
+    ok = True
+
+    def W(bar, parity, phase):
+        nonlocal ok
+        if ok:
+            ok = yield Wait(bar, parity, phase)
+        return ok
 
     def first_s(i, k, kpos, nkv_i):
-        yield Wait(st.q_full[i], k & 1, k)
-        yield Wait(st.k_full[kpos % ST], (kpos // ST) & 1, kpos // ST)
+        if not (yield from W(st.q_full[i], k & 1, k)):
+            return False
+        if not (yield from W(st.k_full[kpos % ST], (kpos // ST) & 1, kpos // ST)):
+            return False
         yield s_mma(st, i, k, 0, kpos % ST, kpos)
         yield Commit("mma", st.s_full[i])
         if i == 1:
             yield Commit("mma", st.k_empty[kpos % ST])
         if nkv_i == 1:
             yield Commit("mma", st.q_empty[i])
+        return True
 
     for k, (n0, n1) in enumerate(cfg.units):
+        if not ok:
+            break
         nxt = cfg.units[k + 1] if (cfg.separate_p and k + 1 < n_units) else (0, 0)
-        if not early[0]:
-            yield from first_s(0, k, kc, n0)
-        if not early[1]:
-            yield from first_s(1, k, kc, n1)
+        if not early[0] and not (yield from first_s(0, k, kc, n0)):
+            break
+        if not early[1] and not (yield from first_s(1, k, kc, n1)):
+            break
         early = [False, False]
         for j in range(n1):
             vn, kn = vc + j, kc + j + 1
             vst, vph, kst, kph = vn % ST, (vn // ST) & 1, kn % ST, (kn // ST) & 1
             if cfg.separate_p:
                 if j + 1 < n0:
-                    if cfg.plant != "no_s_free_wait":
-                        yield Wait(st.s_free[0], sf_cnt[0] & 1, sf_cnt[0])
+                    if cfg.plant != "no_s_free_wait" and not (yield from W(st.s_free[0], sf_cnt[0] & 1, sf_cnt[0])):
+                        break
                     sf_cnt[0] += 1
-                    yield Wait(st.k_full[kst], kph, kn // ST)
+                    if not (yield from W(st.k_full[kst], kph, kn // ST)):
+                        break
                     yield s_mma(st, 0, k, j + 1, kst, kn)
                     yield Commit("mma", st.s_full[0])
                     if j + 2 == n0:
                         yield Commit("mma", st.q_empty[0])
                 if j + 1 < n1:
-                    yield Wait(st.s_free[1], sf_cnt[1] & 1, sf_cnt[1])
+                    if not (yield from W(st.s_free[1], sf_cnt[1] & 1, sf_cnt[1])):
+                        break
                     sf_cnt[1] += 1
-                    if cfg.causal:
-                        yield Wait(st.k_full[kst], kph, kn // ST)
+                    if cfg.causal and not (yield from W(st.k_full[kst], kph, kn // ST)):
+                        break
                     yield s_mma(st, 1, k, j + 1, kst, kn)
                     yield Commit("mma", st.s_full[1])
                     yield Commit("mma", st.k_empty[kst])
                     if j + 2 == n1:
                         yield Commit("mma", st.q_empty[1])
                 if j < n0:
-                    yield Wait(st.pv_ready[0], pv_cnt[0] & 1, pv_cnt[0])
+                    if not (yield from W(st.pv_ready[0], pv_cnt[0] & 1, pv_cnt[0])):
+                        break
                     pv_cnt[0] += 1
-                    if j == 0 and k > 0:
-                        yield Wait(st.o_free[0], (k - 1) & 1, k - 1)
-                    yield Wait(st.v_full[vst], vph, vn // ST)
+                    if j == 0 and k > 0 and not (yield from W(st.o_free[0], (k - 1) & 1, k - 1)):
+                        break
+                    if not (yield from W(st.v_full[vst], vph, vn // ST)):
+                        break
                     yield pv_mma(st, 0, k, j, vst, vn)
                     yield Commit("mma", st.o_done[0])
                     if j + 1 == n0 and nxt[0] > 0:
-                        yield from first_s(0, k + 1, kc + n1, nxt[0])
+                        if not (yield from first_s(0, k + 1, kc + n1, nxt[0])):
+                            break
                         early[0] = True
-                yield Wait(st.pv_ready[1], pv_cnt[1] & 1, pv_cnt[1])
+                if not (yield from W(st.pv_ready[1], pv_cnt[1] & 1, pv_cnt[1])):
+                    break
                 pv_cnt[1] += 1
-                if j == 0 and k > 0:
-                    yield Wait(st.o_free[1], (k - 1) & 1, k - 1)
-                if cfg.causal:
-                    yield Wait(st.v_full[vst], vph, vn // ST)
+                if j == 0 and k > 0 and not (yield from W(st.o_free[1], (k - 1) & 1, k - 1)):
+                    break
+                if cfg.causal and not (yield from W(st.v_full[vst], vph, vn // ST)):
+                    break
                 yield pv_mma(st, 1, k, j, vst, vn)
                 yield Commit("mma", st.o_done[1])
                 yield Commit("mma", st.v_empty[vst])
                 if j + 1 == n1 and nxt[1] > 0:
-                    yield from first_s(1, k + 1, kc + n1, nxt[1])
+                    if not (yield from first_s(1, k + 1, kc + n1, nxt[1])):
+                        break
                     early[1] = True
                 continue
             # d = 128: P_i(j) lives in S_i, so S_i(j+1) is issued behind PV_i(j)
             if cfg.plant == "s_before_pv" and j + 1 < n0:
-                yield Wait(st.k_full[kst], kph, kn // ST)
+                if not (yield from W(st.k_full[kst], kph, kn // ST)):
+                    break
                 yield s_mma(st, 0, k, j + 1, kst, kn)
             if j < n0:
-                yield Wait(st.pv_ready[0], pv_cnt[0] & 1, pv_cnt[0])
+                if not (yield from W(st.pv_ready[0], pv_cnt[0] & 1, pv_cnt[0])):
+                    break
                 pv_cnt[0] += 1
-                if j == 0 and k > 0:
-                    yield Wait(st.o_free[0], (k - 1) & 1, k - 1)
-                yield Wait(st.v_full[vst], vph, vn // ST)
+                if j == 0 and k > 0 and not (yield from W(st.o_free[0], (k - 1) & 1, k - 1)):
+                    break
+                if not (yield from W(st.v_full[vst], vph, vn // ST)):
+                    break
                 yield pv_mma(st, 0, k, j, vst, vn)
                 yield Commit("mma", st.o_done[0])
             if j + 1 < n0:
                 if cfg.plant != "s_before_pv":
-                    yield Wait(st.k_full[kst], kph, kn // ST)
+                    if not (yield from W(st.k_full[kst], kph, kn // ST)):
+                        break
                     yield s_mma(st, 0, k, j + 1, kst, kn)
                 yield Commit("mma", st.s_full[0])
                 if j + 2 == n0:
                     yield Commit("mma", st.q_empty[0])
-            yield Wait(st.pv_ready[1], pv_cnt[1] & 1, pv_cnt[1])
+            if not (yield from W(st.pv_ready[1], pv_cnt[1] & 1, pv_cnt[1])):
+                break
             pv_cnt[1] += 1
-            if j == 0 and k > 0:
-                yield Wait(st.o_free[1], (k - 1) & 1, k - 1)
-            yield Wait(st.v_full[vst], vph, vn // ST)
+            if j == 0 and k > 0 and not (yield from W(st.o_free[1], (k - 1) & 1, k - 1)):
+                break
+            if not (yield from W(st.v_full[vst], vph, vn // ST)):
+                break
             yield pv_mma(st, 1, k, j, vst, vn)
             yield Commit("mma", st.o_done[1])
             yield Commit("mma", st.v_empty[vst])
             if j + 1 < n1:
-                yield Wait(st.k_full[kst], kph, kn // ST)
+                if not (yield from W(st.k_full[kst], kph, kn // ST)):
+                    break
                 yield s_mma(st, 1, k, j + 1, kst, kn)
                 yield Commit("mma", st.s_full[1])
                 yield Commit("mma", st.k_empty[kst])
@@ -348,19 +425,27 @@ def mma_issuer(st: State):
                     yield Commit("mma", st.q_empty[1])
         kc += n1
         vc += n1
-    yield Commit("mma", st.drain)
-    yield Wait(st.drain, 0, 0)
+    # all MMAs complete before tensor memory is released
+    if cfg.plant != "no_mma_drain":
+        yield Commit("mma", st.drain)
+        yield Wait(st.drain, 0, 0, drain=True)
+    yield from teardown(st)
 
 
 def softmax_warp(st: State, i: int, q: int):
     """Warp q of softmax warpgroup i: rows 32q..32q+31 of query tile i."""
     cfg, BS = st.cfg, st.cfg.bias_stages
     s_cnt = od_cnt = bcnt = 0
+    ok = True
     for k in range(len(cfg.units)):
+        if not ok:
+            break
         nkv = nkv_of(cfg, k, i)
         for j in range(nkv):
-            yield Wait(st.s_full[i], s_cnt & 1, s_cnt)
+            ok = yield Wait(st.s_full[i], s_cnt & 1, s_cnt)
             s_cnt += 1
+            if not ok:
+                break
 
             def read_s(s, k=k, j=j):
                 s.expect(f"softmax{i}.{q} reads S{i}({k},{j})", s.tS[i][q], ("S", k, j))
@@ -369,7 +454,9 @@ def softmax_warp(st: State, i: int, q: int):
                 yield Arrive(st.s_free[i], 32)
             if BS:
                 bst = bcnt % BS
-                yield Wait(st.bias_full[i][bst], (bcnt // BS) & 1, bcnt // BS)
+                ok = yield Wait(st.bias_full[i][bst], (bcnt // BS) & 1, bcnt // BS)
+                if not ok:
+                    break
 
                 def read_b(s, k=k, j=j, bst=bst):
                     s.expect(f"softmax{i}.{q} reads bias", s.sBias[i][bst], (k, j))
@@ -387,9 +474,9 @@ def softmax_warp(st: State, i: int, q: int):
                     yield Do("alpha", put_alpha)
                     yield Arrive(st.sm2corr[i], 32)
                 if cfg.plant != "no_o_done_wait":
-                    yield Wait(st.o_done[i], od_cnt & 1, od_cnt)
+                    ok = yield Wait(st.o_done[i], od_cnt & 1, od_cnt)
                 od_cnt += 1
-                if cfg.plant != "alpha_before_o_done":
+                if ok and cfg.plant != "alpha_before_o_done":
                     yield Do("alpha", put_alpha)
                     yield Arrive(st.sm2corr[i], 32)
 
@@ -398,17 +485,25 @@ def softmax_warp(st: State, i: int, q: int):
                     s.tP[i][q] = ("P", k, j)
                 else:
                     s.tS[i][q] = ("P", k, j)
-            yield Do("st P", write_p)
+            if ok:
+                yield Do("st P", write_p)
+            if not ok:
+                break
             yield Arrive(st.pv_ready[i], 32)
+        if not ok:
+            break
         if cfg.separate_p:
             od_cnt += 1
         if k > 0 and cfg.plant != "stats_no_o_free_wait":
-            yield Wait(st.o_free[i], (k - 1) & 1, k - 1)
+            ok = yield Wait(st.o_free[i], (k - 1) & 1, k - 1)
+            if not ok:
+                break
 
         def put_stats(s, k=k):
             s.stats[k & 1][i][q] = k
         yield Do("stats", put_stats)
         yield Arrive(st.stats_full[i], 32)
+    yield from teardown(st)
 
 
 def correction_warp(st: State, q: int):
@@ -416,20 +511,32 @@ def correction_warp(st: State, q: int):
     cfg = st.cfg
     c_cnt, st_cnt, od_cnt = [0, 0], [0, 0], [0, 0]
     n_units = len(cfg.units)
+    ok = True
+
+    def WS(bar, counters, i):
+        nonlocal ok
+        if ok:
+            ok = yield Wait(bar, counters[i] & 1, counters[i])
+        counters[i] += 1
+        return ok
+
     for k, (n0, n1) in enumerate(cfg.units):
-        for j in range(n1):
+        if not ok:
+            break
+        j = 0
+        while ok and j < n1:
             for i in range(2):
                 if j >= (n1 if i else n0):
                     continue
                 if j > 0:
-                    yield Wait(st.sm2corr[i], c_cnt[i] & 1, c_cnt[i])
-                    c_cnt[i] += 1
+                    if not (yield from WS(st.sm2corr[i], c_cnt, i)):
+                        break
 
                     def read_alpha(s, k=k, j=j, i=i):
                         s.expect(f"correction.{q} reads alpha{i}", s.alpha[j & 1][i][q], (k, j))
                     yield Do("alpha", read_alpha)
-                    yield Wait(st.o_done[i], od_cnt[i] & 1, od_cnt[i])
-                    od_cnt[i] += 1
+                    if not (yield from WS(st.o_done[i], od_cnt, i)):
+                        break
 
                     def rescale(s, k=k, j=j, i=i):
                         o = s.tO[i][q]
@@ -442,12 +549,15 @@ def correction_warp(st: State, q: int):
                         yield Arrive(st.pv_ready[i], 32)
                 elif k == 0:
                     yield Arrive(st.pv_ready[i], 32)
+            j += 1
+        if not ok:
+            break
         has_next = k + 1 < n_units
         for i in range(2):
-            yield Wait(st.stats_full[i], st_cnt[i] & 1, st_cnt[i])
-            st_cnt[i] += 1
-            yield Wait(st.o_done[i], od_cnt[i] & 1, od_cnt[i])
-            od_cnt[i] += 1
+            if not (yield from WS(st.stats_full[i], st_cnt, i)):
+                break
+            if not (yield from WS(st.o_done[i], od_cnt, i)):
+                break
             last = (n1 if i else n0) - 1
 
             def epilogue(s, k=k, i=i, last=last):
@@ -459,28 +569,37 @@ def correction_warp(st: State, q: int):
             yield Arrive(st.o_free[i], 32)
             if has_next:
                 yield Arrive(st.pv_ready[i], 32)
+    yield from teardown(st)
 
 
 def kernel_roles(st: State) -> dict:
-    roles = {"tma": producer(st), "mma": mma_issuer(st), "corr": None}
+    roles = {"tma": producer(st), "mma": mma_issuer(st)}
     for i in range(2):
         for q in range(4):
             roles[f"softmax{i}.{q}"] = softmax_warp(st, i, q)
     for q in range(4):
         roles[f"corr.{q}"] = correction_warp(st, q)
-    del roles["corr"]
     return roles
 
 
 # ---------------------------------------------------------------------------------------- scheduler
-def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_steps: int = 2_000_000) -> int:
-    """Executes the roles under one random schedule; returns the number of actions taken."""
+def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_steps: int = 2_000_000,
+        info: dict = None) -> int:
+    """Executes the roles under one random schedule; returns the number of actions taken.
+
+    A bounded wait (not a drain) returns True once its phase has completed; it returns False
+    (leaving the phase unobserved) when the abort flag is up and the phase has not completed,
+    or when it is the wait named by cfg.timeout, which also raises the flag.  Drain waits only
+    return once their phase completed.  When the teardown barrier completes, no TMA load and no
+    tensor-core operation may still be in flight."""
     rng = random.Random(seed)
     st = state_cls(cfg)
     roles = make_roles(st)
     current = {}                    # role -> pending action
+    bounded_waits = {}              # role -> bounded waits reached so far
     for name, gen in roles.items():
         current[name] = next(gen, None)
+        bounded_waits[name] = 0
     fifos: dict[str, list] = {}     # tcgen05 thread -> [Issue | Commit]
     tma: list = []
     trace: list = []
@@ -489,6 +608,9 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
         tail = "\n  ".join(trace[-25:])
         raise ProtocolError(f"{msg}\n  seed {seed}, units {cfg.units}\n  last actions:\n  {tail}")
 
+    def timed_out(name, a):
+        return (not a.drain) and cfg.timeout == (name, bounded_waits[name])
+
     steps = 0
     while True:
         choices = []
@@ -496,7 +618,8 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
             if a is None:
                 continue
             if isinstance(a, Wait) and not a.bar.try_wait(a.parity):
-                continue
+                if a.drain or not (st.abort or timed_out(name, a)):
+                    continue
             choices.append(("role", name))
         for th, f in fifos.items():
             if f:
@@ -509,11 +632,14 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
                 desc = ", ".join(f"{n} waits {a.bar.name} phase {a.phase} (completed {a.bar.completed})"
                                  for n, a in blocked.items())
                 fail(f"deadlock: {desc}")
+            if info is not None:
+                info["aborted"] = st.abort
             return steps
         kind, key = rng.choice(choices)
         steps += 1
         if steps > max_steps:
             fail("step limit")
+        result = None
         try:
             if kind == "tc":
                 item = fifos[key].pop(0)
@@ -534,10 +660,23 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
             if isinstance(a, Wait):
                 if a.parity & 1 != a.phase & 1:
                     fail(f"{key}: waits {a.bar.name} with parity {a.parity} for phase {a.phase}")
-                if a.bar.completed != a.phase + 1:
-                    fail(f"{key}: wait on {a.bar.name} for phase {a.phase} returned with "
-                         f"{a.bar.completed} phases completed (parity aliasing)")
-                trace.append(f"{key}: waited {a.bar.name} phase {a.phase}")
+                forced = timed_out(key, a)
+                if not a.drain:
+                    bounded_waits[key] += 1
+                if forced or not a.bar.try_wait(a.parity):
+                    st.abort = True
+                    result = False
+                    trace.append(f"{key}: wait on {a.bar.name} phase {a.phase} gives up")
+                else:
+                    if a.bar.completed != a.phase + 1:
+                        fail(f"{key}: wait on {a.bar.name} for phase {a.phase} returned with "
+                             f"{a.bar.completed} phases completed (parity aliasing)")
+                    result = True
+                    trace.append(f"{key}: waited {a.bar.name} phase {a.phase}")
+                    if a.bar is st.teardown and (any(fifos.values()) or tma):
+                        pending = [i.name if isinstance(i, Issue) else "commit " + i.bar.name
+                                   for f in fifos.values() for i in f] + [t.name for t in tma]
+                        fail(f"teardown with asynchronous work in flight: {pending}")
             elif isinstance(a, Arrive):
                 trace.append(f"{key}: arrive {a.bar.name} x{a.n}")
                 a.bar.arrive(a.n)
@@ -556,4 +695,7 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
             if "last actions" in str(e):
                 raise
             fail(str(e))
-        current[key] = next(roles[key], None)
+        try:
+            current[key] = roles[key].send(result)
+        except StopIteration:
+            current[key] = None

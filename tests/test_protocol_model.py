@@ -1,13 +1,15 @@
 """The forward kernel's mbarrier protocol, executed as a model under random schedules (CPU).
 
-tests/protocol_model.py restates the barrier protocol of attn_fwd_kernel.cuh (one actor per
-warp, asynchronous tensor-core and TMA work, version-tagged buffers).  These tests run it over
-the kernel's configurations (separate P columns at d <= 64 or P inside S at d = 128, causal or
-not, K/V ring depths 2-4, staged bias tiles) and over random unit sequences, including units of
-a single key tile and causal units whose second query tile reaches one more key tile than the
-first.  Every run must finish without a stale read, a parity-aliased wait or a deadlock.  The
-last test plants protocol mistakes of the kinds a change to the kernel could make and checks
-that the model finds each of them.
+tests/protocol_model.py restates the barrier protocol of attn_fwd_kernel.cuh: one actor per
+warp, asynchronous tensor-core and TMA work, version-tagged buffers, and the abort path of the
+bounded waits.  These tests run it over the kernel's configurations (separate P columns at
+d <= 64 or P inside S at d = 128, causal or not, K/V ring depths 2-4, staged bias tiles) and
+over random unit sequences, including units of a single key tile and causal units whose second
+query tile reaches one more key tile than the first.  Every run must finish without a stale
+read, a parity-aliased wait or a deadlock.  With a timeout forced at any wait of any role,
+every role must still reach the teardown, with no TMA load or tensor-core operation in flight
+when tensor memory is freed.  Other tests plant protocol mistakes of the kinds a change to the
+kernel could make and check that the model finds each of them.
 """
 import random
 
@@ -50,6 +52,42 @@ def test_single_tile_units_back_to_back():
         cfg = pm.Config(separate_p=rep % 2 == 0, causal=True, stages=3,
                         units=[(1, 1 + (rep + u) % 2) for u in range(6)])
         pm.run(cfg, seed=rep)
+
+
+ROLES = ["tma", "mma"] + [f"softmax{i}.{q}" for i in range(2) for q in range(4)] + [f"corr.{q}" for q in range(4)]
+
+
+@pytest.mark.parametrize("sep,causal,stages,bias", [(True, True, 3, 0), (True, False, 4, 2), (True, True, 3, 1),
+                                                    (False, True, 2, 0), (False, False, 2, 0)])
+def test_a_timeout_at_any_wait_drains_and_exits(sep, causal, stages, bias):
+    # every role, every one of its first bounded waits: the wait gives up (as after the kernel's
+    # clock64 limit), the abort flag goes up, and every role must still leave its loops, the
+    # producer and the MMA warp must drain, and nothing may be in flight at teardown
+    units = [(2, 3), (1, 1), (3, 3)] if causal else [(2, 2), (1, 1), (3, 3)]
+    aborted = 0
+    for role in ROLES:
+        for idx in range(10):
+            info = {}
+            cfg = pm.Config(separate_p=sep, causal=causal, stages=stages, bias_stages=bias, units=units,
+                            timeout=(role, idx))
+            pm.run(cfg, seed=idx, info=info)
+            aborted += info["aborted"]
+    assert aborted >= 100, aborted
+
+
+@pytest.mark.parametrize("plant", ["no_tma_drain", "no_mma_drain"])
+def test_model_finds_a_missing_drain(plant):
+    for rep in range(200):
+        rng = random.Random(rep)
+        cfg = pm.Config(separate_p=rep % 2 == 0, causal=True, stages=3 if rep % 2 == 0 else 2,
+                        units=pm.random_units(rng, True, 2, max_tiles=3), plant=plant,
+                        timeout=(rng.choice(ROLES), rng.randint(0, 4)))
+        try:
+            pm.run(cfg, seed=rep)
+        except pm.ProtocolError as e:
+            assert "in flight" in str(e)
+            return
+    pytest.fail(f"{plant!r} went unnoticed")
 
 
 PLANTS = {
@@ -99,4 +137,5 @@ def test_model_barriers_match_the_kernel_source():
             model[name] = bars[0].count
         elif isinstance(val, pm.Barrier):
             model[name] = val.count
+    model.pop("teardown")         # the kernel's __syncthreads before tensor memory is freed
     assert found == model
