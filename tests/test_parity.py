@@ -116,6 +116,26 @@ def test_strided_views():
     assert_close_to_oracle(out_buf.transpose(1, 2), lse, o_ref, l_ref, torch.bfloat16, "strided")
 
 
+def test_evoformer_column_gated_attention():
+    """Column-wise gated self-attention of an Evoformer MSA block (the gated Evoformer variant of
+    the FLASHLIGHT summary, along the other axis): the MSA activations are [R, C, H, d] and each
+    column attends over its R rows, with a sigmoid gate and no pair bias.  The kernel runs on
+    permuted views of the row-major buffers (batch = columns, sequence = rows), no copies."""
+    R, C, H, d = 200, 24, 8, 32
+    g = torch.Generator().manual_seed(12)
+    mk = lambda: torch.randn(R, C, H, d, generator=g).to(torch.bfloat16)
+    qb, kb, vb, gb = mk(), mk(), mk(), mk()
+    dev = torch.device("cuda")
+    col = lambda x: x.permute(1, 2, 0, 3)              # [C, H, R, d]
+    q, k, v, gate = (col(x.to(dev)) for x in (qb, kb, vb, gb))
+    out_buf = torch.zeros(R, C, H, d, device=dev, dtype=torch.bfloat16)
+    _, lse = attn_fwd(q, k, v, gate=gate, causal=False, out=col(out_buf))
+    torch.cuda.synchronize()
+    assert last_device_status() == 0, "a bounded device wait timed out"
+    o_ref, l_ref = sdpa_forward(col(qb), col(kb), col(vb), gate=col(gb))
+    assert_close_to_oracle(col(out_buf), lse, o_ref, l_ref, torch.bfloat16, "evoformer column")
+
+
 @pytest.mark.parametrize("name", ["gpt2_small", "evoformer_row"])
 def test_deterministic(name):
     """Repeated launches give bit-identical results (no atomics; any race in the
