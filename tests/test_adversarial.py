@@ -3,7 +3,6 @@ on every tile, huge magnitudes, -inf biases, one dominant key, identical value
 rows, scale 0 (a closed form), and fully masked rows."""
 import math
 
-import numpy as np
 import pytest
 import torch
 

@@ -1,7 +1,6 @@
 """GPU parity of the score modifications (attn_fwd_ex: ALiBi, logit softcap,
 left window) against the fp64 oracle on the same seeded inputs, every output
 row compared, with the forward's tolerances."""
-import math
 
 import pytest
 import torch

@@ -5,7 +5,6 @@ brute-force tiny case."""
 import math
 
 import numpy as np
-import pytest
 
 from oracle import sdpa_forward, sdpa_varlen_forward
 

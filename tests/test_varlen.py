@@ -4,7 +4,7 @@ import pytest
 import torch
 
 from exact_attention_sdpa_b200 import attn_fwd_varlen, last_device_status
-from exact_attention_sdpa_b200.workloads import WORKLOADS, Workload, make_varlen_inputs
+from exact_attention_sdpa_b200.workloads import WORKLOADS, make_varlen_inputs
 from oracle import sdpa_varlen_forward
 from helpers import assert_close_to_oracle
 
