@@ -130,12 +130,17 @@ def _mutant(kind):
             if p.shape[0] == p.shape[1]:
                 return dq, dk, p @ do
             return dq, dk, dv[::-1]
+        if kind == "no_causal_mask":
+            return real(q, k, v, do, False, scale, offset)
+        if kind == "top_left_alignment":
+            return real(q, k, v, do, causal, scale, 0)
         return real(q, k, v, do, causal, scale, offset)
 
     return grad
 
 
-@pytest.mark.parametrize("kind", ["dq_without_scale", "softmax_jacobian_sign", "dk_from_k", "dv_untransposed"])
+@pytest.mark.parametrize("kind", ["dq_without_scale", "softmax_jacobian_sign", "dk_from_k", "dv_untransposed",
+                                  "no_causal_mask", "top_left_alignment"])
 def test_backward_pins_catch_planted_mistake(kind, monkeypatch):
     monkeypatch.setattr(osdpa, "_grad_rows", _mutant(kind))
     caught = 0

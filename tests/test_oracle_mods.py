@@ -131,6 +131,59 @@ def _mutant(kind):
     return attend
 
 
+def _mutant_scores(kind):
+    """_attend_rows with one mistake in how the modifications meet the scores and the masks."""
+    def attend(qr, k, v, bias_r, gate_r, rows, causal, scale, offset=0, mods=None):
+        s = scale * (qr @ k.T)
+        if bias_r is not None:
+            s = s + bias_r
+        keys = np.arange(k.shape[0])
+        diag = rows[:, None] + (0 if kind in ("alibi_no_offset", "window_no_offset") else offset)
+        if causal and kind == "softcap_after_mask":
+            s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
+        if mods is not None:
+            if mods.get("alibi_slope") is not None:
+                d_al = diag if kind == "alibi_no_offset" else rows[:, None] + offset
+                s = s - mods["alibi_slope"] * np.abs(d_al - keys[None, :])
+            cap = mods.get("softcap", 0.0)
+            if cap and cap > 0:
+                s = cap * np.tanh(s) if kind == "softcap_no_inner_division" else cap * np.tanh(s / cap)
+            w = mods.get("window_left", -1)
+            if w is not None and w >= 0:
+                d_w = diag if kind == "window_no_offset" else rows[:, None] + offset
+                s = np.where(keys[None, :] < d_w - w, -np.inf, s)
+        if causal and kind != "softcap_after_mask":
+            s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
+        m = s.max(axis=1)
+        dead = ~np.isfinite(m) & (m < 0)
+        wts = np.exp(s - np.where(dead, 0.0, m)[:, None])
+        l = wts.sum(axis=1)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            o = np.where(dead[:, None], 0.0, (wts @ v) / l[:, None])
+            lse = np.where(dead, -np.inf, m + np.log(l))
+        if gate_r is not None:
+            o = o * (1.0 / (1.0 + np.exp(-gate_r)))
+        return o, lse
+    return attend
+
+
+@pytest.mark.parametrize("kind", ["none", "alibi_no_offset", "window_no_offset", "softcap_no_inner_division",
+                                  "softcap_after_mask"])
+def test_mod_pins_catch_planted_score_mistake(kind, monkeypatch):
+    monkeypatch.setattr(osdpa, "_attend_rows", _mutant_scores(kind))
+    failed = []
+    for pin in MOD_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(osdpa.sdpa_forward)
+        except (AssertionError, FloatingPointError, ValueError):
+            failed.append(pin.__name__)
+    if kind == "none":          # the scaffold without a mistake is faithful
+        assert not failed, failed
+    else:
+        assert failed, f"no pin caught the planted mistake {kind!r}"
+
+
 @pytest.mark.parametrize("kind", ["alibi_sign", "window_off_by_one", "softcap_before_scale"])
 def test_mod_pins_catch_planted_mistake(kind, monkeypatch):
     monkeypatch.setattr(osdpa, "_attend_rows", _mutant(kind))
