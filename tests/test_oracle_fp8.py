@@ -164,3 +164,54 @@ def test_bound_rejects_a_saturating_configuration():
     qc, kc, vc = (_codes(rng, (1, 1, 4, 16)) for _ in range(3))
     with pytest.raises(AssertionError):
         p_rounding_bound(qc, kc, vc, 1.0, 1.0, 1.0, p_prescale=256.0, threshold_log2=8.0)
+
+
+def _codec_mutant(kind):
+    """e4m3_decode / e4m3_round with one plausible mistake."""
+    import oracle.fp8 as f8
+    real_decode, real_round = f8.e4m3_decode, f8.e4m3_round
+
+    def decode(codes):
+        c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+        out = real_decode(codes)
+        if kind == "exponent_bias_8":
+            out = out / 2.0
+        if kind == "subnormal_scale":
+            sub = ((c >> 3) & 0xF) == 0
+            out = np.where(sub, out * 2.0, out)
+        if kind == "no_nan":
+            out = np.where(np.isnan(out), np.copysign(480.0, np.where(c & 0x80, -1.0, 1.0)), out)
+        return out
+
+    def rnd(x):
+        r = real_round(x)
+        if kind == "ties_away":
+            vals = real_decode(np.arange(0x7F, dtype=np.uint8))
+            a = np.abs(np.asarray(x, dtype=np.float64))
+            mids = (vals[:-1] + vals[1:]) / 2
+            hit = np.isin(a, mids)
+            up = vals[np.clip(np.searchsorted(vals, a), 0, len(vals) - 1)]
+            r = np.where(hit, np.copysign(up, x), r)
+        if kind == "no_saturation":
+            r = np.where(np.abs(np.asarray(x)) > E4M3_MAX, np.nan, r)
+        return r
+    return decode, rnd
+
+
+CODEC_PINS = [test_decode_matches_torch_on_every_code, test_decode_closed_forms, test_round_matches_torch_on_random_values,
+              test_round_ties_go_to_the_even_code, test_round_saturates_at_448]
+
+
+@pytest.mark.parametrize("kind", ["exponent_bias_8", "subnormal_scale", "no_nan", "ties_away", "no_saturation"])
+def test_codec_pins_catch_planted_mistake(kind, monkeypatch):
+    decode, rnd = _codec_mutant(kind)
+    monkeypatch.setitem(globals(), "e4m3_decode", decode)
+    monkeypatch.setitem(globals(), "e4m3_round", rnd)
+    caught = 0
+    for pin in CODEC_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"no pin caught the planted mistake {kind!r}"
