@@ -156,7 +156,7 @@ def barrier(world: int):
 def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
     """The fp64 oracle, as it stands, on a bounded sample of the workload:
     each step computes `rows_per_step` full output rows of one (b, h) head.
-    Returns (TFLOPS over the sampled work, description, cores)."""
+    Returns (TFLOPS over the sampled work, description, cores, mean ms per timed step)."""
     import numpy as np
 
     from oracle import sdpa_rows
@@ -188,7 +188,7 @@ def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
             flops += 4.0 * w.d * vis
     cores = len(os.sched_getaffinity(0))
     sample = f"{rows_per_step} query rows (the last, i.e. heaviest) of one random (b,h) head per step, {steps} steps"
-    return flops / secs / 1e12, sample, cores
+    return flops / secs / 1e12, sample, cores, 1e3 * secs / max(steps, 1)
 
 
 def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
@@ -378,9 +378,10 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:
             return
-        val, sample, cores = cpu_reference(w, args.steps, args.warmup)
+        val, sample, cores, ms = cpu_reference(w, args.steps, args.warmup)
         line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
                 "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
                 "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -480,7 +481,7 @@ def main():
             "clocks": clocks.summary()}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, sample, cores = cpu_reference(w, args.cpu_steps, 1)
+        val, sample, cores, _ = cpu_reference(w, args.cpu_steps, 1)
         line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -63,6 +63,25 @@ def test_reference_arm_prints_from_rank_zero_only():
     assert r.returncode == 0 and r.stdout.strip() == ""
 
 
+def test_reference_arm_line_keeps_the_contract():
+    # rank 0 of the reference arm prints one JSON line with the contract's keys (CPU, seconds)
+    import json
+    env = dict(os.environ)
+    for key in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(key, None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr[-500:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["ms_per_step"] > 0
+    assert line["config"]["workload"] == "n8192_causal"
+    assert set(line["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
 def test_launch_percentiles():
     sys.path.insert(0, ROOT)
     import bench
