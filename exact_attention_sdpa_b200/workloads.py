@@ -86,6 +86,9 @@ WORKLOADS: Dict[str, Workload] = {
                  lengths=(3072, 512, 1911, 4096, 256, 2600, 1024, 3333, 768, 1500, 4000, 2048, 300, 2900, 1200, 3600),
                  description="a ragged batch of 16 sequences of 256-4096 tokens (36,920 in all), H=12 d=64 "
                              "fp16, causal, packed along the token axis"),
+        Workload("n8192_window", B=4, H=12, N=8192, d=64, dtype="fp16", causal=True, seed=8, window_left=1023,
+                 description="the B=4 H=12 N=8192 d=64 fp16 causal sizing with a left (sliding) window of "
+                             "1024 keys per query"),
         Workload("prefill_chunk", B=8, H=12, N=2048, d=64, dtype="fp16", causal=True, seed=5, Nk=8192,
                  description="a 2048-row prefill chunk against an 8192-row KV cache, B=8 H=12 d=64 fp16, "
                              "causal (bottom-right aligned)"),
@@ -143,7 +146,17 @@ def make_varlen_inputs(w: Workload, seed: Optional[int] = None):
 def attention_flops(w: Workload) -> float:
     """The metric's FLOP count: 4*B*H*N^2*d, halved for causal (square problems).  With
     Nk keys: 4*B*H*d times the number of visible (query, key) pairs, N*Nk without causal
-    masking, and with it the pairs j <= i + (Nk - N) (N*Nk - N*(N-1)/2 when N <= Nk)."""
+    masking, and with it the pairs j <= i + (Nk - N) (N*Nk - N*(N-1)/2 when N <= Nk).
+    With a left window w >= 0 (keys j >= i + (Nk - N) - w): the visible pairs, counted exactly."""
+    if w.window_left is not None and w.window_left >= 0 and w.lengths is None:
+        n, nk = w.N, w.n_keys
+        off = nk - n
+        pairs = 0
+        for i in range(n):
+            hi = min(nk - 1, i + off) if w.causal else nk - 1
+            lo = max(0, i + off - w.window_left)
+            pairs += max(0, hi - lo + 1)
+        return 4.0 * w.B * w.H * w.d * pairs
     if w.lengths is not None:
         f = sum(4.0 * w.H * n * n * w.d for n in w.lengths)
         return f / 2.0 if w.causal else f

@@ -48,3 +48,14 @@ def test_alibi_slopes():
     assert alibi_slopes(WORKLOADS["n8192_causal"]) is None
     s = alibi_slopes(WORKLOADS["n8192_alibi_softcap"])
     assert s.shape == (12,) and abs(s[0].item() - 2 ** (-8 / 12)) < 1e-7 and abs(s[-1].item() - 2 ** -8) < 1e-9
+
+
+def test_window_counts_visible_pairs_by_brute_force():
+    for n, nk, causal, wl in [(7, 7, True, 2), (5, 9, True, 3), (9, 4, True, 1), (6, 8, False, 2), (300, 300, True, 63)]:
+        w = Workload("win", B=2, H=3, N=n, d=8, dtype="fp16", causal=causal, seed=0, Nk=nk, window_left=wl)
+        off = nk - n
+        pairs = sum(1 for i in range(n) for j in range(nk)
+                    if j >= i + off - wl and (not causal or j <= i + off))
+        assert attention_flops(w) == 4.0 * 2 * 3 * 8 * pairs
+    big = WORKLOADS["n8192_window"]
+    assert attention_flops(big) == 4.0 * 4 * 12 * 64 * sum(min(i, 1023) + 1 for i in range(8192))
