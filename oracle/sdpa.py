@@ -40,6 +40,10 @@ exponentials shifted by it.  Readings of points the pages leave open:
   c * tanh(s / c); a left window w >= 0 masks keys j < i + (Nk - Nq) - w (a
   sliding window, together with the causal mask a band of w + 1 keys).
 
+* the gradients with score modifications follow from the chain rule: the ALiBi
+  shift and the window mask do not depend on Q or K, and the softcap multiplies
+  dS by its derivative 1 - tanh(s / c)^2.
+
 Inputs of any float dtype are upcast exactly to float64 before any arithmetic.
 Parity: every function is pinned (tests/test_oracle.py, test_oracle_mods.py,
 test_oracle_varlen.py, test_oracle_backward.py, test_oracle_properties.py).
@@ -197,7 +201,7 @@ def sdpa_rows(q, k, v, picks: Sequence[Tuple[int, int, int]], bias=None, gate=No
 # backward
 # ---------------------------------------------------------------------------
 
-def _grad_rows(q, k, v, do, causal, scale, offset):
+def _grad_rows(q, k, v, do, causal, scale, offset, mods=None):
     """Gradients of one (b, h) head without bias or gate, from the definition.
 
     These are the derivatives of Equation (1) of aiinarabic.com
@@ -213,11 +217,29 @@ def _grad_rows(q, k, v, do, causal, scale, offset):
 
     P is formed here with the two-pass softmax of the forward definition (not
     from a saved lse), so the oracle does not depend on the forward under test.
+
+    Score modifications (``mods`` as in _attend_rows, applied in the forward's
+    order): the ALiBi shift and the window mask do not depend on Q or K, so they
+    change only P; the softcap t = c tanh(s / c) has the derivative 1 - tanh(s / c)^2,
+    by which dS is multiplied before dQ and dK are formed (the chain rule).
     """
     s = scale * (q @ k.T)
+    rows = np.arange(q.shape[0])
+    keys = np.arange(k.shape[0])
+    dcap = None
+    if mods is not None:
+        slope = mods.get("alibi_slope")
+        if slope is not None:
+            s = s - slope * np.abs(rows[:, None] + offset - keys[None, :])
+        cap = mods.get("softcap", 0.0)
+        if cap and cap > 0:
+            t = np.tanh(s / cap)
+            s = cap * t
+            dcap = 1.0 - t * t
+        w = mods.get("window_left", -1)
+        if w is not None and w >= 0:
+            s = np.where(keys[None, :] < rows[:, None] + offset - w, -np.inf, s)
     if causal:
-        rows = np.arange(q.shape[0])
-        keys = np.arange(k.shape[0])
         s = np.where(keys[None, :] > rows[:, None] + offset, -np.inf, s)
     m = s.max(axis=1)
     dead = ~np.isfinite(m)
@@ -230,18 +252,22 @@ def _grad_rows(q, k, v, do, causal, scale, offset):
     dv = p.T @ do
     dp = do @ v.T
     ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    if dcap is not None:
+        ds = ds * dcap
     dq = scale * (ds @ k)
     dk = scale * (ds.T @ q)
     return dq, dk, dv
 
 
-def sdpa_backward(q, k, v, do, causal: bool = False, scale: Optional[float] = None
-                  ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+def sdpa_backward(q, k, v, do, causal: bool = False, scale: Optional[float] = None, softcap: float = 0.0,
+                  alibi_slopes=None, window_left: int = -1) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """(dQ, dK, dV) in float64 for O = softmax(scale Q K^T [causal]) V and upstream dO.
 
     q, do: [B,H,Nq,d]; k, v: [B,H,Nk,d]; causal masking aligned as in the forward
-    (key j visible to query i iff j <= i + Nk - Nq).  No bias or gate.
+    (key j visible to query i iff j <= i + Nk - Nq).  No bias or gate.  softcap,
+    alibi_slopes ([H]) and window_left as in sdpa_forward (off by default).
     """
+    alibi_slopes = None if alibi_slopes is None else to_f64(alibi_slopes)
     q, k, v, do = (to_f64(t) for t in (q, k, v, do))
     _check(q, k, v, causal)
     assert do.shape == q.shape
@@ -252,7 +278,8 @@ def sdpa_backward(q, k, v, do, causal: bool = False, scale: Optional[float] = No
     for b in range(B):
         for h in range(H):
             dQ[b, h], dK[b, h], dV[b, h] = _grad_rows(q[b, h], k[b, h], v[b, h], do[b, h], causal, scale,
-                                                      k.shape[2] - Nq)
+                                                      k.shape[2] - Nq,
+                                                      mods=_head_mods(softcap, alibi_slopes, window_left, h))
     return dQ, dK, dV
 
 
