@@ -23,7 +23,8 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_grad_output", "make_varlen_inputs", "alibi_slopes", "attention_flops", "algorithmic_bytes"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_e4m3_inputs", "make_grad_output", "make_varlen_inputs",
+           "alibi_slopes", "attention_flops", "algorithmic_bytes"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -121,6 +122,29 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, Optional[t
     bias = draw(w.H, w.N, w.n_keys) if w.bias else None
     gate = draw(*shape) if w.gate else None
     return {"q": q, "k": k, "v": v, "bias": bias, "gate": gate}
+
+
+def make_e4m3_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, object]:
+    """Inputs for the FP8 forward: q, k, v as e4m3 codes (torch.float8_e4m3fn, CPU) with one
+    power-of-two scale per tensor.
+
+    The fp32 draws are those of make_inputs (same generator, same order q, k, v, times amp).
+    Each tensor's scale is the smallest power of two s with max|x| / s <= 448 (the largest e4m3
+    value), so x / s is exact and torch's round-to-nearest conversion to e4m3 never saturates;
+    element c of the codes stands for c * s.  Returns q, k, v and q_scale, k_scale, v_scale.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    out: Dict[str, object] = {}
+    for name, n in (("q", w.N), ("k", w.n_keys), ("v", w.n_keys)):
+        x = torch.randn(w.B, w.H, n, w.d, generator=g, dtype=torch.float32)
+        if w.amp != 1.0:
+            x.mul_(w.amp)
+        amax = float(x.abs().max())
+        s = 2.0 ** math.ceil(math.log2(amax / 448.0)) if amax > 0 else 1.0
+        out[name] = (x / s).to(torch.float8_e4m3fn)
+        out[name + "_scale"] = s
+    return out
 
 
 def make_varlen_inputs(w: Workload, seed: Optional[int] = None):

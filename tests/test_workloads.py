@@ -3,7 +3,7 @@ counts (no GPU): the counts are written from the definitions the bench states.""
 import torch
 
 from exact_attention_sdpa_b200.workloads import (WORKLOADS, Workload, algorithmic_bytes, alibi_slopes,
-                                                 attention_flops, make_grad_output, make_inputs,
+                                                 attention_flops, make_e4m3_inputs, make_grad_output, make_inputs,
                                                  make_varlen_inputs)
 
 
@@ -59,3 +59,22 @@ def test_window_counts_visible_pairs_by_brute_force():
         assert attention_flops(w) == 4.0 * 2 * 3 * 8 * pairs
     big = WORKLOADS["n8192_window"]
     assert attention_flops(big) == 4.0 * 4 * 12 * 64 * sum(min(i, 1023) + 1 for i in range(8192))
+
+
+def test_e4m3_inputs_are_seeded_scaled_codes_of_the_same_draws():
+    import math
+    w = Workload("f8", B=1, H=2, N=40, d=64, dtype="bf16", causal=True, seed=21, Nk=72)
+    a, b = make_e4m3_inputs(w), make_e4m3_inputs(w)
+    g = torch.Generator().manual_seed(21)
+    for name, n in (("q", 40), ("k", 72), ("v", 72)):
+        c = a[name]
+        assert c.dtype == torch.float8_e4m3fn and c.shape == (1, 2, n, 64)
+        assert torch.equal(c.view(torch.uint8), b[name].view(torch.uint8))
+        s = a[name + "_scale"]
+        assert s > 0 and math.log2(s) == round(math.log2(s))             # a power of two
+        x = torch.randn(1, 2, n, 64, generator=g, dtype=torch.float32).double()   # the same draws
+        y = c.to(torch.float64) * s
+        assert not torch.isnan(y).any() and float(y.abs().max()) <= 448 * s
+        # e4m3 rounding: within 2^-4 relative for normal values, 2^-10 * s absolute below 2^-6 * s
+        err = (y - x).abs()
+        assert bool((err <= torch.maximum(x.abs() * 2.0 ** -4, torch.full_like(x, 2.0 ** -10 * s))).all())
