@@ -195,3 +195,28 @@ def test_mod_pins_catch_planted_mistake(kind, monkeypatch):
         except (AssertionError, FloatingPointError, ValueError):
             caught += 1
     assert caught >= 1, f"no pin caught the planted mistake {kind!r}"
+
+
+@pytest.mark.parametrize("causal,nq,nk", [(True, 7, 7), (True, 5, 11), (False, 6, 9), (True, 9, 4)])
+def test_alibi_and_window_equal_their_explicit_bias(causal, nq, nk):
+    # the modifications are defined as score terms; written out as an additive bias matrix
+    # (-slope_h |i + Nk - Nq - j|, and -inf left of the window) the plain forward must agree
+    rng = np.random.default_rng(900 + nq * nk)
+    q, k, v = rng.standard_normal((2, 2, nq, 8)), rng.standard_normal((2, 2, nk, 8)), rng.standard_normal((2, 2, nk, 8))
+    slopes = np.array([0.4, 0.05])
+    off = nk - nq
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    alibi_bias = -slopes[:, None, None] * np.abs(i + off - j)[None]              # [H, Nq, Nk]
+    o, lse = sdpa_forward(q, k, v, causal=causal, scale=0.7, alibi_slopes=slopes)
+    ob, lb = sdpa_forward(q, k, v, bias=alibi_bias, causal=causal, scale=0.7)
+    np.testing.assert_allclose(o, ob, atol=1e-13)
+    np.testing.assert_allclose(lse, lb, atol=1e-13)
+    w = 2
+    win_bias = np.where(j < i + off - w, -np.inf, 0.0)[None].repeat(2, axis=0)   # [H, Nq, Nk]
+    o, lse = sdpa_forward(q, k, v, causal=causal, scale=0.7, window_left=w)
+    ob, lb = sdpa_forward(q, k, v, bias=win_bias, causal=causal, scale=0.7)
+    np.testing.assert_allclose(o, ob, atol=1e-13)
+    np.testing.assert_array_equal(np.isfinite(lse), np.isfinite(lb))
+    fin = np.isfinite(lb)
+    np.testing.assert_allclose(lse[fin], lb[fin], atol=1e-13)
