@@ -184,7 +184,10 @@ def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
         if step >= warmup:
             secs += dt
             nk, off = w.n_keys, w.n_keys - w.N
-            vis = sum(min(nk, max(0, i + off + 1)) if w.causal else nk for (_, _, i) in picks)
+            # visible keys of row i: up to i + off (causal) or all, from i + off - window (left window)
+            vis = sum(max(0, (min(nk, i + off + 1) if w.causal else nk) -
+                          (max(0, i + off - w.window_left) if w.window_left >= 0 else 0))
+                      for (_, _, i) in picks)
             flops += 4.0 * w.d * vis
     cores = len(os.sched_getaffinity(0))
     sample = f"{rows_per_step} query rows (the last, i.e. heaviest) of one random (b,h) head per step, {steps} steps"
