@@ -35,6 +35,8 @@ KERNEL_SOURCES = ["exact_attention_sdpa_b200/csrc/attn_fwd_kernel.cuh", "exact_a
 
 
 def kernel_source_hash() -> str:
+    """First 16 hex digits of the SHA-256 of the kernel sources; ncu traffic is reported only
+    for the hash it was captured on."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
@@ -43,6 +45,8 @@ def kernel_source_hash() -> str:
 
 
 def load_peaks():
+    """(peaks, source): the measured HBM copy rate and bf16 GEMM rates of this machine's GPUs when
+    MEASURED_PEAKS.json exists, else the earlier measurements used as fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
@@ -148,6 +152,7 @@ def whole_job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> f
 
 
 def barrier(world: int):
+    """A process-group barrier when more than one rank runs (no-op for a single process)."""
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -354,6 +359,7 @@ def run_varlen(args, w, config):
 
 
 def main():
+    """Parse the contract's arguments and print one JSON line (see the module docstring)."""
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

@@ -87,6 +87,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
 
 
 def status_string(code: int) -> str:
+    """The library's text for a status code (attn_status_string)."""
     return load_library().attn_status_string(code).decode()
 
 
@@ -282,11 +283,15 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[torch.
 
 
 def last_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronises `stream` (default: the current one) and returns ATTN_ERR_TIMEOUT if any kernel
+    of the library gave up a bounded wait since the last call, else ATTN_OK, and clears the word
+    (ATTN_ERR_CUDA if the synchronisation or the read fails)."""
     s = (stream or torch.cuda.current_stream()).cuda_stream
     return load_library().attn_last_device_status(s)
 
 
 def set_wait_limit(cycles: int):
+    """Clock cycles a device-side wait polls before it gives up (applies to later launches)."""
     load_library().attn_set_wait_limit(int(cycles))
 
 
@@ -296,4 +301,5 @@ def debug_inject_stall(enable: bool):
 
 
 def version() -> str:
+    """The library's version string."""
     return load_library().attn_version().decode()

@@ -18,6 +18,7 @@ ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def nvcc_path() -> str:
+    """The nvcc to use: $NVCC, then the one on PATH, then /usr/local/cuda/bin/nvcc."""
     for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
         if cand and os.path.exists(cand):
             return cand
@@ -32,6 +33,7 @@ def _inputs():
 
 
 def is_stale() -> bool:
+    """True when libattn.so is missing or older than any CUDA source or public header."""
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
@@ -39,6 +41,8 @@ def is_stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libattn.so in the package directory for sm_100a (when stale or forced); returns its
+    path.  Raises RuntimeError with nvcc's output if the compilation fails."""
     if not force and not is_stale():
         return LIB
     cmd = [nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",

@@ -49,6 +49,7 @@ class Workload:
 
     @property
     def n_keys(self) -> int:
+        """Key rows: Nk when given, else N."""
         return self.N if self.Nk is None else self.Nk
 
     @property
@@ -58,9 +59,11 @@ class Workload:
 
     @property
     def torch_dtype(self) -> torch.dtype:
+        """The torch dtype of the 16-bit inputs and outputs."""
         return {"fp16": torch.float16, "bf16": torch.bfloat16}[self.dtype]
 
     def with_(self, **kw) -> "Workload":
+        """A copy with the given fields replaced."""
         return dataclasses.replace(self, **kw)
 
 
