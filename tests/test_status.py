@@ -38,6 +38,44 @@ def test_timeout_is_reported_and_context_survives():
     assert_close_to_oracle(o, lse, o_ref, l_ref, torch.float16, "after-timeout")
 
 
+VARIANTS = {
+    # the same stall and abort path in the other kernel builds: staged pair bias + gate at d = 32,
+    # P inside S at d = 128, and the score-modification build (softcap + left window)
+    "d32_bias_gate": (Workload("st32", B=2, H=2, N=300, d=32, dtype="bf16", causal=False, seed=6, bias=True,
+                               gate=True), {}),
+    "d128_causal": (Workload("st128", B=1, H=2, N=600, d=128, dtype="bf16", causal=True, seed=7), {}),
+    "d64_mods": (Workload("stm", B=1, H=2, N=700, d=64, dtype="fp16", causal=True, seed=8),
+                 {"softcap": 20.0, "window_left": 150}),
+}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+def test_timeout_in_other_builds(variant):
+    from helpers import padded
+    w, mods = VARIANTS[variant]
+    inp = make_inputs(w)
+    dev = torch.device("cuda")
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    bias = None if inp["bias"] is None else padded(inp["bias"], dev)
+    gate = None if inp["gate"] is None else inp["gate"].to(dev)
+    assert last_device_status() == nat.ATTN_OK
+    try:
+        set_wait_limit(1 << 21)
+        nat.debug_inject_stall(True)
+        attn_fwd(q, k, v, bias=bias, gate=gate, causal=w.causal, scale=w.scale, **mods)
+        assert last_device_status() == nat.ATTN_ERR_TIMEOUT
+    finally:
+        nat.debug_inject_stall(False)
+        set_wait_limit(DEFAULT_LIMIT)
+    o, lse = attn_fwd(q, k, v, bias=bias, gate=gate, causal=w.causal, scale=w.scale, **mods)
+    torch.cuda.synchronize()
+    assert last_device_status() == nat.ATTN_OK
+    o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], bias=inp["bias"], gate=inp["gate"], causal=w.causal,
+                                scale=w.scale, **mods)
+    assert_close_to_oracle(o, lse, o_ref, l_ref, w.torch_dtype, f"after-timeout {variant}")
+
+
 def test_wait_limit_setter_is_host_only():
     # host-side setter; no device work (runs without a GPU)
     nat.load_library()
