@@ -26,7 +26,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 from exact_attention_sdpa_b200.workloads import (WORKLOADS, algorithmic_bytes, alibi_slopes,  # noqa: E402
-                                                 attention_flops, make_inputs)
+                                                 attention_flops, exponential_count, make_inputs)
 
 METRIC = "attention fwd TFLOPS (4BHN²d, /2 causal) and % of B200 dense BF16/FP16 peak"
 UNIT = "TFLOPS"
@@ -74,7 +74,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -254,6 +254,31 @@ def fp32_fma_peak_tflops(sm_mhz: float) -> float:
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
+# NVIDIA's B200 datasheet dense (no 2:4 sparsity) FP16/BF16 tensor-core rate, TFLOP/s
+DATASHEET_DENSE_TFLOPS = 2250.0
+
+
+def mufu_exp_peak(sm_mhz: float) -> float:
+    """Exponentials per second of the special-function units: 148 SMs x 16 per clock."""
+    return 148 * 16 * sm_mhz * 1e6
+
+
+def peak_fractions(value_per_gpu: float, measured_tflops: float) -> dict:
+    """The metric's percentage against the datasheet dense peak, and against the measured GEMM rate."""
+    return {"pct_of_peak": 100.0 * value_per_gpu / DATASHEET_DENSE_TFLOPS,
+            "pct_of_peak_basis": f"datasheet dense FP16/BF16 {DATASHEET_DENSE_TFLOPS:.0f} TFLOP/s",
+            "pct_of_measured_gemm": 100.0 * value_per_gpu / measured_tflops}
+
+
+def exp_bound(w, mean_launch_ms: float, sm_mhz: float) -> dict:
+    """The special-function-unit bound of a launch: its exponentials at 16 per SM per clock."""
+    n = exponential_count(w)
+    peak = mufu_exp_peak(sm_mhz)
+    return {"exponentials_per_launch": n, "mufu_only_ms": 1e3 * n / peak,
+            "achieved_gexp_s": n / (mean_launch_ms * 1e-3) / 1e9, "peak_gexp_s": peak / 1e9,
+            "frac": (n / (mean_launch_ms * 1e-3)) / peak}
+
+
 def run_bwd(args, w, config):
     """The backward on one GPU: K timed attn_bwd launches (two kernels each) after W warm-ups,
     inputs, O, lse and dO resident.  FLOPs: the usual 2.5x the forward's (five N x N x d
@@ -336,7 +361,7 @@ def run_varlen(args, w, config):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded N(0,1) packed inputs)", "config": dict(config, lengths=list(w.lengths)),
-            "pct_of_peak": 100.0 * value / peak,
+            **peak_fractions(value, peak),
             "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": None,
                          "kernel": "attn_fwd_kernel (one launch per sequence)", "algorithmic_flops_per_launch": flops},
@@ -475,19 +500,34 @@ def main():
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops"]            # burst figure: the kernel is timed alone; fp16 dense rate = bf16's
     achieved = flops / (mean_launch_ms * 1e-3) / 1e12
+    cs = clocks.summary()
+    sm_max = cs["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+    nbytes = algorithmic_bytes(w)
+    hbm = {"achieved_gbs": nbytes / (mean_launch_ms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
+           "frac": nbytes / (mean_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+           "algorithmic_bytes_per_launch": nbytes, "peak_source": f"{peak_src} hbm_gbs"}
+    exps = exp_bound(w, mean_launch_ms, sm_max)
+    if w.d <= 32 and exps["mufu_only_ms"] > 1e3 * flops / (peak * 1e12):
+        # short, narrow heads (the gated Evoformer row attention): the exponentials on the
+        # special-function units bind before the tensor cores (every exponential on MUFU here)
+        roofline = {"bound": "alu", "achieved": exps["achieved_gexp_s"], "peak": exps["peak_gexp_s"],
+                    "unit": "Gexp/s", "frac": exps["frac"],
+                    "peak_source": "MUFU: 148 SMs x 16 exponentials per clock x max SM clock",
+                    "tensor": {"achieved_tflops": achieved, "peak_tflops": peak, "frac": achieved / peak}}
+    else:
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    roofline.update({"traffic": load_traffic(w.name), "kernel": "attn_fwd_kernel",
+                     "mean_launch_ms": mean_launch_ms, "launch_ms_percentiles": launch_percentiles(launch_ms),
+                     "algorithmic_flops_per_launch": flops, "hbm": hbm, "exp": exps})
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs)", "config": config,
-            "pct_of_peak": 100.0 * (value / world) / peak,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "traffic": load_traffic(w.name), "kernel": "attn_fwd_kernel",
-                         "mean_launch_ms": mean_launch_ms,
-                         "launch_ms_percentiles": launch_percentiles(launch_ms),
-                         "algorithmic_flops_per_launch": flops},
+            **peak_fractions(value / world, peak),
+            "roofline": roofline,
             "gpu_launches": args.steps,
             "e2e": e2e,
-            "clocks": clocks.summary()}
+            "clocks": cs}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, sample, cores, _ = cpu_reference(w, args.cpu_steps, 1)

@@ -24,7 +24,7 @@ from typing import Dict, Optional
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_e4m3_inputs", "make_grad_output", "make_varlen_inputs",
-           "alibi_slopes", "attention_flops", "algorithmic_bytes"]
+           "alibi_slopes", "attention_flops", "algorithmic_bytes", "exponential_count"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -197,6 +197,17 @@ def attention_flops(w: Workload) -> float:
         off = nk - n
         pairs = sum(min(nk, max(0, i + off + 1)) for i in range(n))
     return 4.0 * w.B * w.H * w.d * pairs
+
+
+def exponential_count(w: Workload) -> float:
+    """Exponentials the method must evaluate at least once: one per visible (query, key) pair
+    (the softmax weights) plus one per output element when a sigmoid gate is applied."""
+    pairs = attention_flops(w) / (4.0 * w.d)
+    if w.lengths is not None:
+        rows = sum(w.lengths) * w.H
+    else:
+        rows = w.B * w.H * w.N
+    return pairs + (rows * w.d if w.gate else 0.0)
 
 
 def algorithmic_bytes(w: Workload) -> int:

@@ -65,6 +65,26 @@ def test_workload_full_size_sampled(name):
     assert_close_to_oracle(o_s, l_s, o_ref, l_ref, w.torch_dtype, name)
     # every output row (not only the sampled ones) is finite
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    # whole heads, every row and column: the first and last (b, h) of the launch and random
+    # others (every head has units in every wave of the persistent schedule)
+    n_whole = WHOLE_HEADS.get(name, 0)
+    if n_whole:
+        rng = np.random.default_rng(1)
+        heads = [(0, 0), (w.B - 1, w.H - 1)]
+        while len(heads) < n_whole:
+            bh = (int(rng.integers(w.B)), int(rng.integers(w.H)))
+            if bh not in heads:
+                heads.append(bh)
+        o_c, l_c = o.cpu(), lse.cpu()
+        for b, h in heads:
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            o_ref, l_ref = sdpa_forward(inp["q"][sl], inp["k"][sl], inp["v"][sl], causal=w.causal, scale=w.scale)
+            assert_close_to_oracle(o_c[sl], l_c[sl], o_ref, l_ref, w.torch_dtype, f"{name} head ({b},{h})")
+
+
+# heads compared in full at the full-size workloads (the oracle takes ~1 s per N=8192 head
+# and ~15 s per N=32768 head on a 16-core host)
+WHOLE_HEADS = {"n8192_causal": 8, "long_wide": 2, "prefill_chunk": 2}
 
 
 SWEEP = []
