@@ -23,7 +23,7 @@ ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
 
 # every function include/attn.h declares
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
-            "attn_debug_inject_stall", "attn_version")
+            "attn_debug_inject_stall", "attn_debug_exp2", "attn_version")
 
 
 class AttnTensor(ctypes.Structure):
@@ -79,6 +79,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_set_wait_limit.restype = None
         lib.attn_debug_inject_stall.argtypes = [ctypes.c_int]
         lib.attn_debug_inject_stall.restype = None
+        lib.attn_debug_exp2.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                        ctypes.c_void_p]
+        lib.attn_debug_exp2.restype = ctypes.c_int
         lib.attn_version.argtypes = []
         lib.attn_version.restype = ctypes.c_char_p
         if path is None:
@@ -298,6 +301,20 @@ def set_wait_limit(cycles: int):
 def debug_inject_stall(enable: bool):
     """Test hook: later launches time out on purpose (see include/attn.h)."""
     load_library().attn_debug_inject_stall(int(bool(enable)))
+
+
+EXP2_FMA_PIPE, EXP2_MUFU, EXP2_CUDA_EXP2F = 0, 1, 2
+
+
+def debug_exp2(x: torch.Tensor, mode: int) -> torch.Tensor:
+    """Test hook: 2^x on the device with one of the kernel's exponentials (attn_debug_exp2);
+    ``x`` is a contiguous float32 CUDA tensor.  Returns a new tensor (the stream is not synchronised)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("debug_exp2 takes a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    s = torch.cuda.current_stream(x.device).cuda_stream
+    _check(load_library().attn_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), int(mode), s))
+    return y
 
 
 def version() -> str:

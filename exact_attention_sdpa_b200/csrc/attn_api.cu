@@ -452,9 +452,42 @@ attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const att
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Test hook of attn_debug_exp2: thread t evaluates elements 2t and 2t + 1 (one pair, as the
+// softmax does) with the exponential selected by `mode`.
+__global__ void exp2_probe_kernel(const float* x, float* y, int64_t n, int mode) {
+    const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const bool two = i + 1 < n;
+    const float x0 = x[i], x1 = two ? x[i + 1] : 0.f;
+    float y0, y1;
+    if (mode == ATTN_EXP2_FMA_PIPE) {
+        attn::ex2_emu2(y0, y1, x0, x1);
+    } else if (mode == ATTN_EXP2_MUFU) {
+        y0 = attn::sm100::ex2_approx(x0);
+        y1 = attn::sm100::ex2_approx(x1);
+    } else {
+        y0 = exp2f(x0);
+        y1 = exp2f(x1);
+    }
+    y[i] = y0;
+    if (two) y[i + 1] = y1;
+}
+
 }  // namespace
 
 extern "C" {
+
+attn_status_t attn_debug_exp2(const float* x, float* y, int64_t n, int mode, cudaStream_t stream) {
+    if (n < 0 || mode < ATTN_EXP2_FMA_PIPE || mode > ATTN_EXP2_CUDA_EXP2F) return ATTN_ERR_INVALID_ARG;
+    if (n == 0) return ATTN_OK;
+    if (x == nullptr || y == nullptr) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) & 3u) != 0 || (reinterpret_cast<uintptr_t>(y) & 3u) != 0)
+        return ATTN_ERR_INVALID_ARG;
+    const int64_t blocks = ((n + 1) / 2 + 255) / 256;
+    if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    exp2_probe_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, y, n, mode);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                             const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,

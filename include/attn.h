@@ -245,6 +245,28 @@ void attn_set_wait_limit(uint64_t cycles);
  */
 void attn_debug_inject_stall(int enable);
 
+/*
+ * attn_debug_exp2 -- test hook: evaluates, on the device, one of the base-2
+ * exponentials the forward kernel's softmax uses, so that each can be checked
+ * against the exact value and against CUDA's exp2f.  Not part of the
+ * attention computation (the pages define no such call).
+ *
+ *   x, y    device float arrays of n elements (4-byte aligned); y[i] = 2^x[i].
+ *           Elements are taken in pairs (2t, 2t + 1), as the softmax does.
+ *   mode    ATTN_EXP2_FMA_PIPE: the kernel's FMA-pipe 2^x (range reduction with a
+ *           round-down add, a cubic for 2^f on [0, 1), the integer part added to
+ *           the exponent field).  Stated bound: relative error <= 7.5e-5 for
+ *           x in (-126, 8]; x <= -126 gives a value <= 2^-126 (flushed later).
+ *           ATTN_EXP2_MUFU: ex2.approx.ftz.f32 on the special-function unit.
+ *           ATTN_EXP2_CUDA_EXP2F: CUDA's exp2f (the comparison reference).
+ *
+ * Returns ATTN_ERR_INVALID_ARG for n < 0, an unknown mode, or (n > 0) a null or
+ * misaligned pointer; ATTN_ERR_CUDA if the launch fails.  Asynchronous on
+ * `stream`; allocates nothing.
+ */
+enum { ATTN_EXP2_FMA_PIPE = 0, ATTN_EXP2_MUFU = 1, ATTN_EXP2_CUDA_EXP2F = 2 };
+attn_status_t attn_debug_exp2(const float* x, float* y, int64_t n, int mode, cudaStream_t stream);
+
 /* The library version as "major.minor.patch" (static string). */
 const char* attn_version(void);
 
