@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -17,6 +18,11 @@ namespace {
 using attn::FwdParams;
 
 __device__ unsigned int g_status_word;
+__device__ unsigned int g_status_read;   // the word's value at the last read-and-clear
+
+// Reads the status word and clears it in one atomic exchange, ordered after the kernels
+// already enqueued on the stream it runs on.
+__global__ void status_exchange_kernel() { g_status_read = atomicExch(&g_status_word, 0u); }
 
 uint64_t g_wait_limit = 1ull << 32;
 int g_inject_stall = 0;
@@ -40,6 +46,14 @@ bool overlaps(const attn_tensor_t* a, const attn_tensor_t* b) {
     return a0 < b1 && b0 < a1;
 }
 
+// A plain byte range [p, p + n) against a tensor's span.
+bool overlaps_bytes(const void* p, size_t n, const attn_tensor_t* t) {
+    if (p == nullptr || t == nullptr || n == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(p), a1 = a0 + n;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(t->data), b1 = b0 + span_bytes(t);
+    return a0 < b1 && b0 < a1;
+}
+
 // Common checks of a 16-bit tensor of rank `ndim`: positive shape, unit inner
 // stride, other strides positive multiples of 8 elements, 16-byte aligned data.
 attn_status_t check_tensor(const attn_tensor_t* t, int ndim) {
@@ -53,6 +67,16 @@ attn_status_t check_tensor(const attn_tensor_t* t, int ndim) {
         if (t->shape[i] > 1 && t->stride[i] == 0) return ATTN_ERR_INVALID_ARG;
     }
     if ((reinterpret_cast<uintptr_t>(t->data) & 15u) != 0) return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+
+// A packed [T, H, d] tensor of a ragged batch: non-negative strides, unit inner stride, data
+// present (span_bytes and the overlap checks read the strides).
+attn_status_t check_packed(const attn_tensor_t* t) {
+    if (t->data == nullptr) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (t->shape[i] <= 0 || t->stride[i] < 0) return ATTN_ERR_INVALID_ARG;
+    if (t->stride[2] != 1) return ATTN_ERR_INVALID_ARG;
     return ATTN_OK;
 }
 
@@ -141,29 +165,25 @@ bool encode_bias_map(CUtensorMap* map, const attn_tensor_t* b) {
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
-int l2_bytes() {
+// A device attribute of the current device, cached per device.  Host threads may call
+// concurrently: the cache entries are atomics (a race only repeats the same query).
+int cached_attribute(cudaDeviceAttr attr, std::atomic<int> (&cache)[64]) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    static int sizes[64] = {0};
-    if (sizes[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev) != cudaSuccess) return 0;
-        sizes[dev] = n;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, attr, dev) != cudaSuccess) return 0;
+        cache[dev].store(v, std::memory_order_relaxed);
     }
-    return sizes[dev];
+    return v;
 }
 
-int sm_count() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    static int counts[64] = {0};
-    if (counts[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        counts[dev] = n;
-    }
-    return counts[dev];
-}
+std::atomic<int> g_l2_bytes[64];
+std::atomic<int> g_sm_count[64];
+
+int l2_bytes() { return cached_attribute(cudaDevAttrL2CacheSize, g_l2_bytes); }
+
+int sm_count() { return cached_attribute(cudaDevAttrMultiProcessorCount, g_sm_count); }
 
 struct Maps {
     CUtensorMap q, k, v, bias;
@@ -544,6 +564,7 @@ attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, co
     if (batch < 0 || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
     const int64_t Tq = q->shape[0], Tk = k->shape[0], H = q->shape[1];
+    attn_status_t st0 = ATTN_OK;
     if (cu_seqlens_q[0] != 0 || cu_seqlens_k[0] != 0 || cu_seqlens_q[batch] != Tq || cu_seqlens_k[batch] != Tk)
         return ATTN_ERR_INVALID_ARG;
     for (int32_t b = 0; b < batch; ++b) {
@@ -552,6 +573,18 @@ attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, co
         if (nq > 0 && nk == 0) return ATTN_ERR_INVALID_ARG;     // queries with no key at all
     }
     if (Tq == 0 || H == 0) return ATTN_OK;
+    // the packed tensors as wholes: O must not overlap any input row of any sequence, and lse
+    // ([H, Tq] fp32) must overlap none of the tensors
+    if ((st0 = check_packed(q)) != ATTN_OK || (st0 = check_packed(k)) != ATTN_OK ||
+        (st0 = check_packed(v)) != ATTN_OK || (st0 = check_packed(out)) != ATTN_OK)
+        return st0;
+    if (overlaps(out, q) || overlaps(out, k) || overlaps(out, v)) return ATTN_ERR_INVALID_ARG;
+    if (lse != nullptr) {
+        const size_t lse_bytes = static_cast<size_t>(H * Tq) * sizeof(float);
+        if (overlaps_bytes(lse, lse_bytes, q) || overlaps_bytes(lse, lse_bytes, k) ||
+            overlaps_bytes(lse, lse_bytes, v) || overlaps_bytes(lse, lse_bytes, out))
+            return ATTN_ERR_INVALID_ARG;
+    }
     // each sequence: a [1, H, n, d] view of the packed [T, H, d] tensors (strides in elements);
     // every check of attn_fwd runs on the first sequence's views before anything is launched
     auto view = [](const attn_tensor_t* t, int64_t row0, int64_t n) {
@@ -610,6 +643,11 @@ attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
             if (overlaps(outs[a], outs[b])) return ATTN_ERR_INVALID_ARG;
     }
     const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
+    {   // lse ([B, H, N] fp32, read) must not overlap a gradient the kernels write
+        const size_t lse_bytes = static_cast<size_t>(B * H * N) * sizeof(float);
+        for (int a = 0; a < 3; ++a)
+            if (overlaps_bytes(lse, lse_bytes, outs[a])) return ATTN_ERR_INVALID_ARG;
+    }
     if (B * H > 65535) return ATTN_ERR_UNSUPPORTED;
 
     attn::bwd::BwdParams p;
@@ -647,12 +685,12 @@ const char* attn_status_string(attn_status_t status) {
 
 attn_status_t attn_last_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
-    unsigned int* ptr = status_word_ptr();
-    if (ptr == nullptr) return ATTN_ERR_CUDA;
+    status_exchange_kernel<<<1, 1, 0, stream>>>();
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     unsigned int v = 0;
-    if (cudaMemcpy(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
-    const unsigned int zero = 0;
-    if (cudaMemcpy(ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(&v, g_status_read, sizeof(v), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
     return (v & attn::kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
 }
 

@@ -144,8 +144,10 @@ attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const 
  *
  * Layout rules as attn_fwd (unit inner stride, other strides multiples of 16
  * bytes, 16-byte aligned data).  A sequence with no query rows is skipped; one
- * with query rows but no key rows is ATTN_ERR_INVALID_ARG.  Every sequence is
- * checked before the first launch.  This version launches the fused kernel
+ * with query rows but no key rows is ATTN_ERR_INVALID_ARG.  The packed out
+ * must not overlap q, k or v anywhere (not only within one sequence), and lse's
+ * H*Tq floats must not overlap any of the four: ATTN_ERR_INVALID_ARG.  Every
+ * sequence is checked before the first launch.  This version launches the fused kernel
  * once per non-empty sequence, in order, on `stream`.
  */
 attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
@@ -203,7 +205,8 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
  *                            the dtype); none may overlap an input or another.
  *
  * Layout rules and errors as attn_fwd; additionally ATTN_ERR_INVALID_ARG for a
- * missing lse, dout, dq, dk or dv, a shape mismatch or an overlap, and
+ * missing lse, dout, dq, dk or dv, a shape mismatch or an overlap (lse's
+ * B*H*N floats included: they must not overlap dq, dk or dv), and
  * ATTN_ERR_UNSUPPORTED for B*H > 65535.  Asynchronous on `stream` (two kernel
  * launches); allocates nothing.
  */
@@ -216,11 +219,17 @@ attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
 const char* attn_status_string(attn_status_t status);
 
 /*
- * attn_last_device_status -- synchronises `stream`, then reads and clears the
- * device status word of the current device.  Kernels bound every wait on an
- * mbarrier; a wait that gives up records ATTN_ERR_TIMEOUT there (and the
- * kernel returns without hanging).  Returns ATTN_OK, ATTN_ERR_TIMEOUT, or
- * ATTN_ERR_CUDA if synchronising or reading failed.
+ * attn_last_device_status -- reads and clears the device status word of the
+ * current device in one atomic exchange enqueued on `stream` (after the kernels
+ * already enqueued there), then synchronises `stream`.  Kernels bound every
+ * wait on an mbarrier; a wait that gives up records ATTN_ERR_TIMEOUT there
+ * (and the kernel returns without hanging).  The word is DEVICE-WIDE: every
+ * launch of the library on that device, on any stream, shares it.  A timeout
+ * of a kernel still running on another stream may therefore be reported by
+ * this call, or by a later one, instead of the caller whose launch it was;
+ * callers that run the library on several streams and need per-call status
+ * must serialise their reads.  Returns ATTN_OK, ATTN_ERR_TIMEOUT, or
+ * ATTN_ERR_CUDA if the exchange, the read or the synchronisation failed.
  */
 attn_status_t attn_last_device_status(cudaStream_t stream);
 

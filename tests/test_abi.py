@@ -315,6 +315,32 @@ def test_varlen_argument_checks(lib):
     assert nat.attn_fwd_varlen_raw(e, e, e.clone(), z, z, True, 0.1, e.clone(), None, 0) == nat.ATTN_OK
 
 
+def test_varlen_aliasing_across_sequences(lib):
+    """O of one sequence must not overlap Q, K or V rows of another; lse overlaps nothing."""
+    buf = torch.zeros(24, 2, 64, dtype=torch.float16)
+    q, o_other = buf[:10], buf[10:20]                    # disjoint: fine
+    k = torch.zeros(12, 2, 64, dtype=torch.float16)
+    cq = torch.tensor([0, 4, 10], dtype=torch.int32)
+    ck = torch.tensor([0, 5, 12], dtype=torch.int32)
+    v = torch.zeros_like(k)
+    call = lambda q_, o_, lse=None: nat.attn_fwd_varlen_raw(q_, k, v, cq, ck, True, 0.1, o_, lse, 0)
+    # out's rows 4..9 (sequence 1) land on q's rows of the same buffer shifted by 6: sequence 0's out
+    # rows and sequence 1's q rows overlap only across sequences
+    o_shift = buf[6:16]
+    assert call(buf[:10], o_shift) == nat.ATTN_ERR_INVALID_ARG
+    lse_bad = buf.view(-1).view(torch.float32)[:2 * 10]   # lse aliasing q's storage
+    assert call(q, o_other, lse_bad) == nat.ATTN_ERR_INVALID_ARG
+
+
+def test_backward_lse_must_not_overlap_gradients(lib):
+    q, k, v, o = _qkv()
+    do, dk, dv = (torch.zeros_like(q) for _ in range(3))
+    dq = torch.zeros_like(q)
+    lse_in_dq = dq.view(-1).view(torch.float32)[:2 * 64]
+    r = nat.attn_bwd_raw(q, k, v, o, lse_in_dq, do, False, 0.125, dq, dk, dv, 0)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+
+
 C_CLIENT = r"""
 #include <stdio.h>
 #include <string.h>
