@@ -7,7 +7,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
@@ -596,22 +598,76 @@ attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, co
         x.stride[0] = n * t->stride[0]; x.stride[1] = t->stride[1]; x.stride[2] = t->stride[0]; x.stride[3] = t->stride[2];
         return x;
     };
-    const int64_t lse_layout[2] = {0, Tq};
-    for (int pass = 0; pass < 2; ++pass) {        // pass 0: validate every sequence; pass 1: launch
-        for (int32_t b = 0; b < batch; ++b) {
-            const int64_t q0 = cu_seqlens_q[b], nq = cu_seqlens_q[b + 1] - q0;
-            const int64_t k0 = cu_seqlens_k[b], nk = cu_seqlens_k[b + 1] - k0;
-            if (nq == 0) continue;
-            attn_tensor_t vq = view(q, q0, nq), vk = view(k, k0, nk), vv = view(v, k0, nk), vo = view(out, q0, nq);
-            bool empty = false;
-            attn_status_t st = validate_fwd(&vq, &vk, &vv, nullptr, nullptr, scale, &vo, lse, &empty);
-            if (st != ATTN_OK) return st;
-            if (pass == 1) {
-                st = fwd_impl(&vq, &vk, &vv, nullptr, nullptr, causal, scale, nullptr, &vo,
-                              lse == nullptr ? nullptr : lse + q0, lse_layout, stream);
-                if (st != ATTN_OK) return st;
-            }
+    std::vector<int32_t> order;                    // non-empty sequences, every one checked first
+    for (int32_t b = 0; b < batch; ++b) {
+        const int64_t q0 = cu_seqlens_q[b], nq = cu_seqlens_q[b + 1] - q0;
+        const int64_t k0 = cu_seqlens_k[b], nk = cu_seqlens_k[b + 1] - k0;
+        if (nq == 0) continue;
+        attn_tensor_t vq = view(q, q0, nq), vk = view(k, k0, nk), vv = view(v, k0, nk), vo = view(out, q0, nq);
+        bool empty = false;
+        attn_status_t st = validate_fwd(&vq, &vk, &vv, nullptr, nullptr, scale, &vo, lse, &empty);
+        if (st != ATTN_OK) return st;
+        order.push_back(b);
+    }
+    if (order.empty()) return ATTN_OK;
+    // heaviest sequences first (query rows x visible keys), in launches of up to kMaxSeq sequences
+    auto work = [&](int32_t b) {
+        const double nq = cu_seqlens_q[b + 1] - cu_seqlens_q[b], nk = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+        return causal ? nq * (nk - 0.5 * nq) : nq * nk;
+    };
+    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return work(a) > work(b); });
+    // packed [1, H, T, d] views of the whole tensors: one tensor map each for every sequence
+    attn_tensor_t pq = view(q, 0, Tq), pk = view(k, 0, Tk), pv = view(v, 0, Tk), po = view(out, 0, Tq);
+    Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!encode_qkv_map(&maps.q, &pq) || !encode_qkv_map(&maps.k, &pk) || !encode_qkv_map(&maps.v, &pv))
+        return ATTN_ERR_CUDA;
+    unsigned int* status = status_word_ptr();
+    if (status == nullptr) return ATTN_ERR_CUDA;
+    const int64_t d = q->shape[2];
+    for (size_t c0 = 0; c0 < order.size(); c0 += attn::kMaxSeq) {
+        const size_t c1 = std::min(order.size(), c0 + attn::kMaxSeq);
+        FwdParams p;
+        std::memset(&p, 0, sizeof(p));
+        p.B = 1;
+        p.H = static_cast<int>(H);
+        p.N = static_cast<int>(Tq);
+        p.Nk = static_cast<int>(Tk);
+        p.num_q_pairs = 1;
+        p.n_kv_tiles = 1;
+        p.head_group = static_cast<int>(H);
+        p.n_seq = static_cast<int>(c1 - c0);
+        int64_t units = 0;
+        for (size_t i = c0; i < c1; ++i) {
+            const int32_t b = order[i];
+            const int s = static_cast<int>(i - c0);
+            p.seq_units[s] = static_cast<int>(units);
+            p.seq_q0[s] = cu_seqlens_q[b];
+            p.seq_k0[s] = cu_seqlens_k[b];
+            p.seq_nq[s] = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+            p.seq_nk[s] = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+            units += H * ((p.seq_nq[s] + attn::kRowsPerUnit - 1) / attn::kRowsPerUnit);
         }
+        if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+        p.seq_units[p.n_seq] = static_cast<int>(units);
+        p.num_units = static_cast<int>(units);
+        p.scale = scale;
+        p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+        p.out = po.data;
+        p.out_sb = po.stride[0];
+        p.out_sh = po.stride[1];
+        p.out_si = po.stride[2];
+        p.lse = lse;
+        p.lse_sb = 0;
+        p.lse_sh = Tq;
+        p.window_left = -1;
+        p.wait_limit = g_wait_limit;
+        p.status = status;
+        p.inject_stall = g_inject_stall;
+        const cudaError_t e = q->dtype == ATTN_BF16
+                                  ? launch_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, false, false, maps, p, stream)
+                                  : launch_dtype<__half>(static_cast<int>(d), causal != 0, false, false, maps, p, stream);
+        if (e != cudaSuccess) return ATTN_ERR_CUDA;
     }
     return ATTN_OK;
 }

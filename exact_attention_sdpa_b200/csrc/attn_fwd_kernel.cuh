@@ -63,6 +63,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f; // log2 domain: rescale only when m grows by > 2^8
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned long long kDrainLimit = 1ull << 32;
+constexpr int kMaxSeq = 64;    // sequences of a ragged batch handled by one launch
 
 struct FwdParams {
     int B, H, N;               // N: query rows
@@ -90,6 +91,12 @@ struct FwdParams {
     unsigned long long wait_limit;
     unsigned int* status;
     int inject_stall;          // test hook: the MMA warp first waits on a barrier nothing arrives on
+    // ragged batch in one launch (n_seq > 0; B = 1 and the tensors are packed [1, H, T, d] views):
+    // sequence s owns query rows seq_q0[s] .. + seq_nq[s] and key rows seq_k0[s] .. + seq_nk[s],
+    // and units seq_units[s] .. seq_units[s + 1] (its query pairs x H, heaviest pairs first)
+    int n_seq;
+    int seq_units[kMaxSeq + 1];
+    int seq_q0[kMaxSeq], seq_k0[kMaxSeq], seq_nq[kMaxSeq], seq_nk[kMaxSeq];
 };
 
 template <int D>
@@ -245,9 +252,13 @@ __device__ __forceinline__ void ex2_emu2(float& y0, float& y1, float x0, float x
     y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
-// One work unit: query rows [q0, q0 + 256) of (b, h); tile i needs key tiles [0, nkv_i).
+// One work unit: query rows [q0, q0 + 256) of (b, h); tile i processes key tiles
+// [kv_lo, kv_lo + nkv_i) (kv_lo > 0 only when a left window skips whole tiles).  The problem's
+// sizes travel with the unit (a ragged batch mixes sequences): N query rows, Nk key rows,
+// off = Nk - N, and the first query / key row of the sequence in the packed tensors.
 struct Unit {
-    int b, h, bh, qp, q0, nkv0, nkv1;
+    int b, h, bh, qp, q0, nkv0, nkv1, kv_lo;
+    int N, Nk, off, q_base, k_base;
 };
 
 // The k-th unit a CTA processes.  Wave k (the k-th unit of every CTA) takes units
@@ -259,32 +270,69 @@ __device__ __forceinline__ int unit_at(int k) {
     return k * G + ((k & 1) ? (G - 1 - b) : b);
 }
 
-template <bool CAUSAL>
+template <bool CAUSAL, bool MODS = false>
 __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
     Unit U;
-    const int BH = p.B * p.H;
-    // Units are taken in groups of `head_group` heads; inside a group the heaviest query
-    // pairs come first (causal load balance).  With head_group = B*H (the default) this is
-    // one group: heaviest pairs of all heads first.  For long sequences whose K/V do not
-    // fit in L2 the host picks a small group, so that the CTAs running at the same time
-    // share the K/V of a few heads in L2 instead of streaming all of them from DRAM.
-    const int G = p.head_group;
-    const int per = G * p.num_q_pairs;
-    const int g = u / per, r = u % per;
-    const int gsize = min(G, BH - g * G);       // the last group may be partial
-    U.qp = p.num_q_pairs - 1 - r / gsize;
-    U.bh = g * G + r % gsize;
-    U.b = U.bh / p.H;
-    U.h = U.bh % p.H;
+    if (p.n_seq > 0) {
+        // ragged batch: the sequence holding unit u is the last s with seq_units[s] <= u
+        int lo = 0, hi = p.n_seq - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.seq_units[mid] <= u) lo = mid;
+            else hi = mid - 1;
+        }
+        const int r = u - p.seq_units[lo];
+        U.N = p.seq_nq[lo];
+        U.Nk = p.seq_nk[lo];
+        U.q_base = p.seq_q0[lo];
+        U.k_base = p.seq_k0[lo];
+        const int nqp = (U.N + kRowsPerUnit - 1) / kRowsPerUnit;
+        U.qp = nqp - 1 - r / p.H;
+        U.h = r % p.H;
+        U.b = 0;
+        U.bh = U.h;
+    } else {
+        // Units are taken in groups of `head_group` heads; inside a group the heaviest query
+        // pairs come first (causal load balance).  With head_group = B*H (the default) this is
+        // one group: heaviest pairs of all heads first.  For long sequences whose K/V do not
+        // fit in L2 the host picks a small group, so that the CTAs running at the same time
+        // share the K/V of a few heads in L2 instead of streaming all of them from DRAM.
+        const int BH = p.B * p.H;
+        const int G = p.head_group;
+        const int per = G * p.num_q_pairs;
+        const int g = u / per, r = u % per;
+        const int gsize = min(G, BH - g * G);       // the last group may be partial
+        U.qp = p.num_q_pairs - 1 - r / gsize;
+        U.bh = g * G + r % gsize;
+        U.b = U.bh / p.H;
+        U.h = U.bh % p.H;
+        U.N = p.N;
+        U.Nk = p.Nk;
+        U.q_base = 0;
+        U.k_base = 0;
+    }
+    U.off = U.Nk - U.N;
+    const int n_kv_tiles = (U.Nk + kBlockN - 1) / kBlockN;
     U.q0 = U.qp * kRowsPerUnit;
     if (CAUSAL) {
         // key tiles up to the one holding the last visible key of the tile's last row; at
         // least one (a tile whose rows all precede every key is processed once, fully masked)
-        const int last0 = U.q0 + kBlockM - 1 + p.causal_off, last1 = last0 + kBlockM;
-        U.nkv0 = last0 < 0 ? 1 : min(p.n_kv_tiles, last0 / kBlockN + 1);
-        U.nkv1 = last1 < 0 ? 1 : min(p.n_kv_tiles, last1 / kBlockN + 1);
+        const int last0 = U.q0 + kBlockM - 1 + U.off, last1 = last0 + kBlockM;
+        U.nkv0 = last0 < 0 ? 1 : min(n_kv_tiles, last0 / kBlockN + 1);
+        U.nkv1 = last1 < 0 ? 1 : min(n_kv_tiles, last1 / kBlockN + 1);
     } else {
-        U.nkv0 = U.nkv1 = p.n_kv_tiles;
+        U.nkv0 = U.nkv1 = n_kv_tiles;
+    }
+    U.kv_lo = 0;
+    if (MODS && p.window_left >= 0) {
+        // left window: key tiles wholly left of the first row's window are skipped.  The unit's
+        // first row has the leftmost window, so both query tiles start at its first key tile (the
+        // second tile may process one tile it masks completely).  kv_lo < nkv_i: the first row's
+        // own diagonal key (or, without causal masking, key Nk - 1) lies at or after it.
+        const int lo_key = U.q0 + U.off - p.window_left;
+        U.kv_lo = lo_key > 0 ? lo_key / kBlockN : 0;
+        U.nkv0 -= U.kv_lo;
+        U.nkv1 -= U.kv_lo;
     }
     return U;
 }
@@ -294,7 +342,7 @@ template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE, bool MOD
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
-                    const FwdParams p) {
+                    const __grid_constant__ FwdParams p) {
     using namespace sm100;
     using C = Cfg<D>;
     constexpr int ST = C::kStages;
@@ -378,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&sh.q_full[i], C::kTileBytes);
                     for (int a = 0; a < C::kNumAtoms; ++a)
                         tma_load_4d(sQ + (i * C::kNumAtoms + a) * C::kAtomBytes, &tm_q, &sh.q_full[i],
-                                    a * C::kAtomCols, U.q0 + i * kBlockM, U.h, U.b, pol_q);
+                                    a * C::kAtomCols, U.q_base + U.q0 + i * kBlockM, U.h, U.b, pol_q);
                 }
                 __syncwarp();
                 ++qc[i];
@@ -395,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int bb = p.bias_sb != 0 ? U.b : 0;
                     for (int half = 0; half < 2; ++half)
                         tma_load_4d(dst + half * BC::kBoxBytes, &tm_bias, &sh.bias_full[i][st],
-                                    j * kBlockN + half * 64, U.q0 + i * kBlockM, U.h, bb, pol_kv);
+                                    (U.kv_lo + j) * kBlockN + half * 64, U.q0 + i * kBlockM, U.h, bb, pol_kv);
                 }
                 __syncwarp();
                 ++bc[i];
@@ -408,13 +456,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&full[st], C::kTileBytes);
                     for (int a = 0; a < C::kNumAtoms; ++a)
                         tma_load_4d(ring + (st * C::kNumAtoms + a) * C::kAtomBytes, map, &full[st],
-                                    a * C::kAtomCols, j * kBlockN, U.h, U.b, pol_kv);
+                                    a * C::kAtomCols, U.k_base + (U.kv_lo + j) * kBlockN, U.h, U.b, pol_kv);
                 }
                 __syncwarp();
                 ++cnt;
             };
             for (int k = 0, u = unit_at(0); ok && u < p.num_units; u = unit_at(++k)) {
-                const Unit U = decode_unit<CAUSAL>(u, p);
+                const Unit U = decode_unit<CAUSAL, MODS>(u, p);
                 load_q(0, U);
                 if (ok) load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, 0, U);
                 if (ok) load_q(1, U);
@@ -513,11 +561,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Issued after that PV, S_i(0) needs no further ordering: its commit covers the PV.
             bool early[2] = {false, false};
             for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
-                const Unit U = decode_unit<CAUSAL>(u, p);
+                const Unit U = decode_unit<CAUSAL, MODS>(u, p);
                 const int u_next = unit_at(uit + 1);
                 int nkv_next[2] = {0, 0};      // 0: no next unit
                 if (C::kSeparateP && u_next < p.num_units) {
-                    const Unit Un = decode_unit<CAUSAL>(u_next, p);
+                    const Unit Un = decode_unit<CAUSAL, MODS>(u_next, p);
                     nkv_next[0] = Un.nkv0;
                     nkv_next[1] = Un.nkv1;
                 }
@@ -635,14 +683,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
         bool ok = true;
         for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
-            const Unit U = decode_unit<CAUSAL>(u, p);
+            const Unit U = decode_unit<CAUSAL, MODS>(u, p);
             const int nkv = i ? U.nkv1 : U.nkv0;
             const int row = U.q0 + i * kBlockM + t;
             const int first_row = U.q0 + i * kBlockM;
             const T* bias_row = nullptr;
             if constexpr (HAS_BIAS)
                 bias_row = reinterpret_cast<const T*>(p.bias) + U.b * p.bias_sb + U.h * p.bias_sh +
-                           static_cast<int64_t>(row < p.N ? row : 0) * p.bias_si;
+                           static_cast<int64_t>(row < U.N ? row : 0) * p.bias_si;
             float m_ref = -INFINITY;                // reference maximum (log2 domain)
             float l = 0.f;
             for (int j = 0; j < nkv; ++j) {
@@ -669,14 +717,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(&sh.s_free[i]);
                     }
                 }
-                const int kv0 = j * kBlockN;
+                const int kv0 = (U.kv_lo + j) * kBlockN;
                 // key tiles past the end, and (causal) tiles reaching past the first row's last key
                 const bool need_mask =
-                    (kv0 + kBlockN > p.Nk) || (CAUSAL && kv0 + kBlockN - 1 > first_row + p.causal_off);
+                    (kv0 + kBlockN > U.Nk) || (CAUSAL && kv0 + kBlockN - 1 > first_row + U.off);
                 float m_tile;   // tile maximum, log2 domain
                 if (fast) {
                     if (need_mask) {
-                        const int lim = CAUSAL ? min(p.Nk - kv0, row + p.causal_off - kv0 + 1) : (p.Nk - kv0);
+                        const int lim = CAUSAL ? min(U.Nk - kv0, row + U.off - kv0 + 1) : (U.Nk - kv0);
 #pragma unroll
                         for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
                     }
@@ -703,13 +751,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 // chunk (c % 64) / 8 of box c / 64, 128-byte swizzle
                                 raw = *reinterpret_cast<const uint4*>(
                                     brow + (c / 64) * BC::kBoxBytes + ((((c % 64) / 8) ^ (t & 7)) << 4));
-                            } else if (row < p.N && kv0 + c + 8 <= p.Nk) {
+                            } else if (row < U.N && kv0 + c + 8 <= U.Nk) {
                                 raw = __ldg(reinterpret_cast<const uint4*>(bias_row + kv0 + c));
                             } else {
                                 T e[8];
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
-                                    e[q] = (row < p.N && kv0 + c + q < p.Nk) ? bias_row[kv0 + c + q] : T(0.f);
+                                    e[q] = (row < U.N && kv0 + c + q < U.Nk) ? bias_row[kv0 + c + q] : T(0.f);
                                 raw = *reinterpret_cast<const uint4*>(e);
                             }
                             const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -733,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (MODS) {
                         if (p.alibi != nullptr) {      // linear distance penalty of this head
                             const float slope = p.alibi[U.h];
-                            const float dist0 = static_cast<float>(row + p.causal_off - kv0);   // exact below 2^24
+                            const float dist0 = static_cast<float>(row + U.off - kv0);   // exact below 2^24
 #pragma unroll
                             for (int c = 0; c < kBlockN; ++c) s[c] = fmaf(-slope, fabsf(dist0 - c), s[c]);
                         }
@@ -744,10 +792,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int c = 0; c < kBlockN; ++c)
                                 s[c] = cap * (1.f - __fdividef(2.f, 1.f + ex2_approx(s[c] * k2)));
                         }
-                        if (p.window_left >= 0) lo = row + p.causal_off - p.window_left - kv0;
+                        if (p.window_left >= 0) lo = row + U.off - p.window_left - kv0;
                     }
                     if (need_mask || (MODS && p.window_left >= 0)) {
-                        const int lim = CAUSAL ? min(p.Nk - kv0, row + p.causal_off - kv0 + 1) : (p.Nk - kv0);
+                        const int lim = CAUSAL ? min(U.Nk - kv0, row + U.off - kv0 + 1) : (U.Nk - kv0);
 #pragma unroll
                         for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim && c >= lo) ? s[c] : -INFINITY;
                     }
@@ -849,7 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return ok;
         };
         for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
-            const Unit U = decode_unit<CAUSAL>(u, p);
+            const Unit U = decode_unit<CAUSAL, MODS>(u, p);
             for (int j = 0; ok && j < U.nkv1; ++j) {
                 for (int i = 0; i < 2; ++i) {
                     if (j >= (i ? U.nkv1 : U.nkv0)) continue;
@@ -890,13 +938,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool has_next = unit_at(uit + 1) < p.num_units;
             for (int i = 0; i < 2; ++i) {
                 const int row = U.q0 + i * kBlockM + t;
-                const bool row_ok = row < p.N;
+                const bool row_ok = row < U.N;
                 T* orow = reinterpret_cast<T*>(p.out) + U.b * p.out_sb + U.h * p.out_sh +
-                          static_cast<int64_t>(row_ok ? row : 0) * p.out_si;
+                          static_cast<int64_t>(U.q_base + (row_ok ? row : 0)) * p.out_si;
                 const T* grow = nullptr;
                 if constexpr (HAS_GATE)
                     grow = reinterpret_cast<const T*>(p.gate) + U.b * p.gate_sb + U.h * p.gate_sh +
-                           static_cast<int64_t>(row_ok ? row : 0) * p.gate_si;
+                           static_cast<int64_t>(U.q_base + (row_ok ? row : 0)) * p.gate_si;
                 constexpr int kPre = (HAS_GATE && D == 32) ? D / 8 : 1;   // gate row prefetched (d = 32)
                 uint4 graw[kPre];
                 if constexpr (HAS_GATE && D == 32) {
@@ -948,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     finish_chunk(r, c);
                 }
                 if (p.lse != nullptr && row_ok)
-                    p.lse[U.b * p.lse_sb + U.h * p.lse_sh + row] =
+                    p.lse[U.b * p.lse_sb + U.h * p.lse_sh + U.q_base + row] =
                         (l > 0.f) ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
             }
         }

@@ -147,8 +147,15 @@ attn_status_t attn_fwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const 
  * with query rows but no key rows is ATTN_ERR_INVALID_ARG.  The packed out
  * must not overlap q, k or v anywhere (not only within one sequence), and lse's
  * H*Tq floats must not overlap any of the four: ATTN_ERR_INVALID_ARG.  Every
- * sequence is checked before the first launch.  This version launches the fused kernel
- * once per non-empty sequence, in order, on `stream`.
+ * sequence is checked before the first launch.  The fused kernel runs once per
+ * 64 non-empty sequences (one launch for batches of up to 64): the sequences'
+ * sizes and offsets travel in the kernel's parameters, heaviest sequences first,
+ * and every CTA of the persistent grid takes units of any sequence.  Tiles are
+ * read through one tensor map over the packed tensors, so a tile that runs past
+ * its sequence's end reads the next sequence's rows: such keys get weight
+ * exactly 0 and such query rows are never stored, but a non-finite value in a
+ * neighbouring sequence's V is multiplied by that zero (as it would be within
+ * one sequence).
  */
 attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t batch, int causal,

@@ -52,3 +52,31 @@ def test_varlen_workload_sampled():
         sub = [0, r1 - r0]
         o_ref, l_ref = sdpa_varlen_forward(inp["q"][r0:r1], inp["k"][r0:r1], inp["v"][r0:r1], sub, sub, causal=True)
         assert_close_to_oracle(o[r0:r1], lse[:, r0:r1], o_ref, l_ref, w.torch_dtype, f"varlen_mix seq {b}")
+
+
+def test_varlen_more_sequences_than_one_launch_holds():
+    """70 sequences: two launches of the fused kernel (64 sequences travel in one launch's
+    parameters), lengths from 1 to 600 with a few empty ones; every row compared."""
+    rng = torch.Generator().manual_seed(7)
+    lens = []
+    for i in range(70):
+        n = int(torch.randint(1, 600, (1,), generator=rng))
+        lens.append((0, 0) if i % 23 == 5 else (n, n))
+    q, k, v, cq, ck = _packed(lens, 2, 64, torch.float16, seed=71)
+    dev = torch.device("cuda")
+    o, lse = attn_fwd_varlen(q.to(dev), k.to(dev), v.to(dev), cq, ck, causal=True)
+    torch.cuda.synchronize()
+    assert last_device_status() == 0
+    o_ref, l_ref = sdpa_varlen_forward(q, k, v, cq.tolist(), ck.tolist(), causal=True)
+    assert_close_to_oracle(o, lse, o_ref, l_ref, torch.float16, "varlen 70 sequences")
+
+
+def test_varlen_single_sequence_equals_plain_forward():
+    from exact_attention_sdpa_b200 import attn_fwd
+    q, k, v, cq, ck = _packed([(777, 777)], 3, 128, torch.bfloat16, seed=72)
+    dev = torch.device("cuda")
+    o, lse = attn_fwd_varlen(q.to(dev), k.to(dev), v.to(dev), cq, ck, causal=True)
+    as4 = lambda x: x.to(dev).transpose(0, 1).unsqueeze(0)
+    o4, lse4 = attn_fwd(as4(q), as4(k), as4(v), causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o4[0].transpose(0, 1)) and torch.equal(lse, lse4[0])
