@@ -249,11 +249,6 @@ def launch_percentiles(ms):
     return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90)}
 
 
-def fp32_fma_peak_tflops(sm_mhz: float) -> float:
-    """FP32 FMA peak of a B200: 148 SMs x 128 FP32 lanes x 2 FLOP per clock."""
-    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
-
-
 # NVIDIA's B200 datasheet dense (no 2:4 sparsity) FP16/BF16 tensor-core rate, TFLOP/s
 DATASHEET_DENSE_TFLOPS = 2250.0
 
@@ -280,9 +275,10 @@ def exp_bound(w, mean_launch_ms: float, sm_mhz: float) -> dict:
 
 
 def run_bwd(args, w, config):
-    """The backward on one GPU: K timed attn_bwd launches (two kernels each) after W warm-ups,
-    inputs, O, lse and dO resident.  FLOPs: the usual 2.5x the forward's (five N x N x d
-    products against two); the kernels recompute S and dP per block, seven products in all."""
+    """The backward on one GPU: K timed attn_bwd calls (three kernels each: D = rowsum(dO * O),
+    dK/dV, dQ) after W warm-ups, inputs, O, lse and dO resident.  FLOPs: the usual 2.5x the
+    forward's (five N x N x d products against two); the kernels recompute S and dP in both
+    the dK/dV and the dQ kernel, seven products in all, on the tensor cores."""
     from exact_attention_sdpa_b200 import attn_bwd, attn_fwd, load_library
     from exact_attention_sdpa_b200.workloads import make_grad_output
     load_library()
@@ -312,16 +308,89 @@ def run_bwd(args, w, config):
     flops = 2.5 * attention_flops(w)
     value = flops / (ms * 1e-3) / 1e12
     cs = clocks.summary()
-    peak = fp32_fma_peak_tflops(cs["sm_max_mhz"] or 1965.0)
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"]
     line = {"metric": "attention bwd TFLOPS (2.5 x forward FLOPs)", "value": value, "unit": UNIT, "n_gpus": 1,
             "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs and dO)",
             "config": dict(config, **{"pass": "backward"}),
-            "roofline": {"bound": "alu", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
-                         "peak_source": "FP32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock",
-                         "traffic": None, "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
+            **peak_fractions(value, peak),
+            "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "traffic": None, "kernel": "bwd_prep_kernel + bwd_dkdv_kernel + bwd_dq_kernel",
                          "algorithmic_flops_per_launch": flops},
-            "gpu_launches": 2 * steps, "e2e": None, "clocks": cs}
+            "gpu_launches": 3 * steps, "e2e": None, "clocks": cs}
+    print(json.dumps(line), flush=True)
+
+
+def run_fp8(args, w, config):
+    """The forward on e4m3 inputs (attn_fwd_fp8) on one GPU: K timed launches after W warm-ups,
+    inputs (q, k and V transposed) resident.  FLOPs as the 16-bit forward's; the roofline is the
+    measured bf16 GEMM rate times the nominal e4m3 / bf16 ratio of the tensor cores (2)."""
+    from exact_attention_sdpa_b200 import load_library
+    from exact_attention_sdpa_b200 import _native as nat
+    from exact_attention_sdpa_b200.workloads import make_e4m3_inputs
+    assert not (w.bias or w.gate or w.softcap > 0 or w.alibi or w.window_left >= 0 or w.lengths), \
+        "the FP8 forward takes the plain problem only"
+    lib = load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_e4m3_inputs(w)
+    q, k = inp["q"].to(dev), inp["k"].to(dev)
+    B, H, Nk, d = inp["v"].shape
+    vbuf = torch.zeros(B, H, d, (Nk + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    vbuf[..., :Nk] = inp["v"].view(torch.uint8).transpose(-1, -2).to(dev)
+    vt = vbuf[..., :Nk].view(torch.float8_e4m3fn)
+    out = torch.empty(q.shape, device=dev, dtype=torch.float16)
+    lse = torch.empty(q.shape[:-1], device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+    views = [nat.make_view(t) for t in (q, k, vt, out)]
+    refs = [ctypes.byref(x) for x in views]
+    status = []
+
+    def step():
+        r = lib.attn_fwd_fp8(refs[0], refs[1], refs[2], float(inp["q_scale"]), float(inp["k_scale"]),
+                             float(inp["v_scale"]), int(w.causal), float(w.scale), refs[3], lse.data_ptr(),
+                             stream.cuda_stream)
+        if r != 0:
+            status.append(r)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if status:
+        raise RuntimeError(f"attn_fwd_fp8 returned status {status[0]}")
+    ms = t0.elapsed_time(t1) / args.steps
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_launch_ms = statistics.mean(launch_ms)
+    flops = attention_flops(w)
+    value = flops / (ms * 1e-3) / 1e12
+    achieved = flops / (mean_launch_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = 2.0 * peaks["bf16_tflops"]
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic (seeded N(0,1) inputs as e4m3 codes with power-of-two scales)",
+            "config": dict(config, dtype="e4m3 in, fp16 out", v_layout="transposed [B, H, d, Nk]"),
+            "pct_of_peak": 100.0 * value / (2.0 * DATASHEET_DENSE_TFLOPS),
+            "pct_of_peak_basis": f"datasheet dense FP8 {2.0 * DATASHEET_DENSE_TFLOPS:.0f} TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3 / bf16 ratio)",
+                         "traffic": None, "kernel": "attn_fwd_kernel (e4m3)", "mean_launch_ms": mean_launch_ms,
+                         "launch_ms_percentiles": launch_percentiles(launch_ms),
+                         "algorithmic_flops_per_launch": flops},
+            "gpu_launches": args.steps, "e2e": None, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
 
 
@@ -396,6 +465,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-staged end-to-end leg (profiling runs)")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward (attn_bwd) on the workload instead of the forward")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the e4m3 forward (attn_fwd_fp8) on the workload's shape instead")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     flops = attention_flops(w)
@@ -424,6 +495,8 @@ def main():
 
     if args.bwd:
         return run_bwd(args, w, config)
+    if args.fp8:
+        return run_fp8(args, w, config)
     if w.lengths is not None:
         return run_varlen(args, w, config)
     world, rank, local = dist_setup(args.gpus)
@@ -488,6 +561,14 @@ def main():
         raise RuntimeError(f"attn_fwd returned status {status[0]}")
     total_ms = t_start.elapsed_time(t_end)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
+    # host time of one C-ABI call (argument checks, tensor-map encoding, launch), outside the
+    # timed region: calls enqueued back to back, the device left to drain afterwards
+    n_host = 50
+    h0 = time.perf_counter()
+    for _ in range(n_host):
+        step()
+    host_us = 1e6 * (time.perf_counter() - h0) / n_host
+    torch.cuda.synchronize()
     ms_per_step = dist_max(total_ms / args.steps, world)
     mean_launch_ms = statistics.mean(launch_ms)
     value = whole_job_tflops(world, flops, ms_per_step)
@@ -526,6 +607,7 @@ def main():
             **peak_fractions(value / world, peak),
             "roofline": roofline,
             "gpu_launches": args.steps,
+            "host_us_per_call": host_us,
             "e2e": e2e,
             "clocks": cs}
 

@@ -19,10 +19,10 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libattn.so")
 
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
-ATTN_F16, ATTN_BF16, ATTN_F32 = 0, 1, 2
+ATTN_F16, ATTN_BF16, ATTN_F32, ATTN_E4M3 = 0, 1, 2, 3
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_bwd", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_fwd_fp8", "attn_bwd", "attn_bwd_ex", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
             "attn_debug_inject_stall", "attn_debug_exp2", "attn_version")
 
 
@@ -68,9 +68,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p,
                                       P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_host.restype = ctypes.c_int
+        lib.attn_fwd_fp8.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int,
+                                     ctypes.c_float, P, ctypes.c_void_p, ctypes.c_void_p]
+        lib.attn_fwd_fp8.restype = ctypes.c_int
         lib.attn_bwd.argtypes = [P, P, P, P, ctypes.c_void_p, P, ctypes.c_int, ctypes.c_float, P, P, P,
                                  ctypes.c_void_p]
         lib.attn_bwd.restype = ctypes.c_int
+        lib.attn_bwd_ex.argtypes = [P, P, P, P, ctypes.c_void_p, P, ctypes.c_int, ctypes.c_float,
+                                    ctypes.POINTER(AttnMods), P, P, P, ctypes.c_void_p]
+        lib.attn_bwd_ex.restype = ctypes.c_int
         lib.attn_status_string.argtypes = [ctypes.c_int]
         lib.attn_status_string.restype = ctypes.c_char_p
         lib.attn_last_device_status.argtypes = [ctypes.c_void_p]
@@ -99,7 +105,8 @@ def _check(code: int):
         raise AttnError(code, status_string(code))
 
 
-_DT = {torch.float16: ATTN_F16, torch.bfloat16: ATTN_BF16, torch.float32: ATTN_F32}
+_DT = {torch.float16: ATTN_F16, torch.bfloat16: ATTN_BF16, torch.float32: ATTN_F32,
+       torch.float8_e4m3fn: ATTN_E4M3}
 
 
 def make_view(t: Optional[torch.Tensor]) -> Optional[AttnTensor]:
@@ -194,21 +201,60 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     return out, lse
 
 
-def attn_bwd_raw(q, k, v, out, lse, dout, causal: bool, scale: float, dq, dk, dv, stream: int) -> int:
-    """Direct call of attn_bwd with torch tensors; returns the status code."""
+def attn_fwd_fp8_raw(q, k, v_t, q_scale: float, k_scale: float, v_scale: float, causal: bool, scale: float, out,
+                     lse, stream: int) -> int:
+    """Direct call of attn_fwd_fp8 with torch tensors; returns the status code."""
+    lib = load_library()
+    vq, vk, vv, vo = (make_view(t) for t in (q, k, v_t, out))
+    return lib.attn_fwd_fp8(_ref(vq), _ref(vk), _ref(vv), float(q_scale), float(k_scale), float(v_scale),
+                            int(bool(causal)), float(scale), _ref(vo), None if lse is None else lse.data_ptr(), stream)
+
+
+def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v_t: torch.Tensor, q_scale: float = 1.0, k_scale: float = 1.0,
+                 v_scale: float = 1.0, causal: bool = False, scale: Optional[float] = None,
+                 out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The forward on e4m3 inputs (include/attn.h, attn_fwd_fp8): q [B, H, N, d], k [B, H, Nk, d]
+    and v_t = V transposed [B, H, d, Nk] as CUDA torch.float8_e4m3fn tensors (d in {64, 128}),
+    element x meaning x * its tensor's scale.  Returns (out [B, H, N, d] in out_dtype, lse)."""
+    if not q.is_cuda:
+        raise ValueError("attn_fwd_fp8 takes CUDA tensors")
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if out is None:
+        out = torch.empty(q.shape, device=q.device, dtype=out_dtype)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(attn_fwd_fp8_raw(q, k, v_t, q_scale, k_scale, v_scale, causal, scale, out, lse, s))
+    return out, lse
+
+
+def attn_bwd_raw(q, k, v, out, lse, dout, causal: bool, scale: float, dq, dk, dv, stream: int,
+                 softcap: float = 0.0, alibi_slopes: Optional[torch.Tensor] = None, window_left: int = -1) -> int:
+    """Direct call of attn_bwd (attn_bwd_ex when a score modification is on); returns the status code."""
     lib = load_library()
     vq, vk, vv, vo, vdo, vdq, vdk, vdv = (make_view(t) for t in (q, k, v, out, dout, dq, dk, dv))
-    return lib.attn_bwd(_ref(vq), _ref(vk), _ref(vv), _ref(vo), None if lse is None else lse.data_ptr(), _ref(vdo),
+    lse_p = None if lse is None else lse.data_ptr()
+    if softcap != 0.0 or alibi_slopes is not None or window_left >= 0:
+        mods = AttnMods(None if alibi_slopes is None else alibi_slopes.data_ptr(), float(softcap), int(window_left))
+        return lib.attn_bwd_ex(_ref(vq), _ref(vk), _ref(vv), _ref(vo), lse_p, _ref(vdo), int(bool(causal)),
+                               float(scale), ctypes.byref(mods), _ref(vdq), _ref(vdk), _ref(vdv), stream)
+    return lib.attn_bwd(_ref(vq), _ref(vk), _ref(vv), _ref(vo), lse_p, _ref(vdo),
                         int(bool(causal)), float(scale), _ref(vdq), _ref(vdk), _ref(vdv), stream)
 
 
 def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
              dout: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
-             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+             stream: Optional[torch.cuda.Stream] = None, softcap: float = 0.0,
+             alibi_slopes: Optional[torch.Tensor] = None,
+             window_left: int = -1) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """(dQ, dK, dV) of attn_fwd (no bias or gate) for the upstream gradient ``dout``.
 
-    ``out`` and ``lse`` are attn_fwd's outputs for the same q, k, v, causal and
-    scale.  CUDA tensors; asynchronous on ``stream`` (default: the current one).
+    ``out`` and ``lse`` are attn_fwd's outputs for the same q, k, v, causal, scale and
+    score modifications (softcap, alibi_slopes, window_left as in attn_fwd).  CUDA
+    tensors; asynchronous on ``stream`` (default: the current one).
     """
     if not q.is_cuda:
         raise ValueError("attn_bwd takes CUDA tensors")
@@ -218,7 +264,8 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     dk = torch.empty_like(k, memory_format=torch.contiguous_format)
     dv = torch.empty_like(v, memory_format=torch.contiguous_format)
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
-    _check(attn_bwd_raw(q, k, v, out, lse, dout, causal, scale, dq, dk, dv, s))
+    _check(attn_bwd_raw(q, k, v, out, lse, dout, causal, scale, dq, dk, dv, s, softcap=softcap,
+                        alibi_slopes=alibi_slopes, window_left=window_left))
     return dq, dk, dv
 
 

@@ -13,7 +13,7 @@
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
-#include "attn_bwd_kernel.cuh"
+#include "attn_bwd_tc.cuh"
 
 namespace {
 
@@ -117,8 +117,8 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// [B, H, N, d] view -> 4-D map with dims {d, N, H, B}, box {min(d,64), 128, 1, 1}
-bool encode_qkv_map(CUtensorMap* map, const attn_tensor_t* t) {
+// [B, H, N, d] view -> 4-D map with dims {d, N, H, B}, box {min(d,64), rows, 1, 1}
+bool encode_qkv_map(CUtensorMap* map, const attn_tensor_t* t, unsigned rows = 128) {
     EncodeTiledFn enc = get_encode_fn();
     if (enc == nullptr) return false;
     const int64_t d = t->shape[3];
@@ -130,13 +130,52 @@ bool encode_qkv_map(CUtensorMap* map, const attn_tensor_t* t) {
     const int64_t sH = stride_or(1, sN * t->shape[2]);
     const int64_t sB = stride_or(0, sH * t->shape[1]);
     const cuuint64_t strides[3] = {(cuuint64_t)(sN * 2), (cuuint64_t)(sH * 2), (cuuint64_t)(sB * 2)};
-    const cuuint32_t box[4] = {(cuuint32_t)(d >= 64 ? 64 : d), 128u, 1u, 1u};
+    const cuuint32_t box[4] = {(cuuint32_t)(d >= 64 ? 64 : d), (cuuint32_t)rows, 1u, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     const CUtensorMapDataType dt =
         t->dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const CUtensorMapSwizzle sw = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     return enc(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// e4m3 [B, H, N, d] view -> 4-D map {d, N, H, B}, box {d, 128, 1, 1}: one swizzle atom per row
+// (64 bytes at d = 64, 128 bytes at d = 128)
+bool encode_e4m3_map(CUtensorMap* map, const attn_tensor_t* t) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (enc == nullptr) return false;
+    const int64_t d = t->shape[3];
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)t->shape[2], (cuuint64_t)t->shape[1],
+                                (cuuint64_t)t->shape[0]};
+    auto stride_or = [&](int i, int64_t fallback) { return t->shape[i] > 1 ? t->stride[i] : fallback; };
+    const int64_t sN = stride_or(2, d);
+    const int64_t sH = stride_or(1, sN * t->shape[2]);
+    const int64_t sB = stride_or(0, sH * t->shape[1]);
+    const cuuint64_t strides[3] = {(cuuint64_t)sN, (cuuint64_t)sH, (cuuint64_t)sB};
+    const cuuint32_t box[4] = {(cuuint32_t)d, 128u, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUtensorMapSwizzle sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, t->data, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// e4m3 V^T [B, H, d, Nk] view -> 4-D map {Nk, d, H, B}, box {128, d, 1, 1}, 128-byte swizzle
+bool encode_e4m3_vt_map(CUtensorMap* map, const attn_tensor_t* t) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (enc == nullptr) return false;
+    const int64_t d = t->shape[2], nk = t->shape[3];
+    const cuuint64_t dims[4] = {(cuuint64_t)nk, (cuuint64_t)d, (cuuint64_t)t->shape[1], (cuuint64_t)t->shape[0]};
+    auto stride_or = [&](int i, int64_t fallback) { return t->shape[i] > 1 ? t->stride[i] : fallback; };
+    const int64_t sD = stride_or(2, (nk + 15) / 16 * 16);
+    const int64_t sH = stride_or(1, sD * d);
+    const int64_t sB = stride_or(0, sH * t->shape[1]);
+    const cuuint64_t strides[3] = {(cuuint64_t)sD, (cuuint64_t)sH, (cuuint64_t)sB};
+    const cuuint32_t box[4] = {128u, (cuuint32_t)d, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, t->data, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bias [H, N, N] or [B, H, N, N] -> 4-D map {keys, rows, H, B}, box {64, 128, 1, 1}, 128-byte swizzle
@@ -191,6 +230,20 @@ struct Maps {
     CUtensorMap q, k, v, bias;
 };
 
+// Raises a kernel's dynamic shared-memory limit once per device.  `done` is the calling
+// launcher's own flag word (one bit per device), so each kernel instantiation is set once;
+// concurrent first calls may both set it, which is harmless.
+template <typename Kern>
+cudaError_t smem_limit_once(Kern kern, int smem, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
 template <typename T, int D, bool CAUSAL, bool BIAS, bool GATE, bool MODS = false>
 cudaError_t launch_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
     auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, BIAS, GATE, MODS>;
@@ -199,11 +252,27 @@ cudaError_t launch_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
     // tensor-memory columns, and a second one would only wait for the first to finish.
     constexpr int smem = attn::BiasCfg<D, BIAS>::kDynBytes > 116 * 1024 ? attn::BiasCfg<D, BIAS>::kDynBytes
                                                                       : 116 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static std::atomic<uint64_t> smem_set{0};
+    cudaError_t e = smem_limit_once(kern, smem, smem_set);
     if (e != cudaSuccess) return e;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
     // persistent: one CTA per SM (tensor memory and registers allow no more)
+    const int grid = p.num_units < sms ? p.num_units : sms;
+    kern<<<grid, attn::kThreads, smem, stream>>>(m.q, m.k, m.v, m.bias, p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, bool CAUSAL>
+cudaError_t launch_fp8_t(const Maps& m, const FwdParams& p, cudaStream_t stream) {
+    auto kern = attn::attn_fwd_kernel<T, D, CAUSAL, false, false, false, true>;
+    constexpr int need = attn::Cfg<D, true>::kDynBytes;
+    constexpr int smem = need > 116 * 1024 ? need : 116 * 1024;     // one CTA per SM (all of TMEM)
+    static std::atomic<uint64_t> smem_set{0};
+    cudaError_t e = smem_limit_once(kern, smem, smem_set);
+    if (e != cudaSuccess) return e;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
     const int grid = p.num_units < sms ? p.num_units : sms;
     kern<<<grid, attn::kThreads, smem, stream>>>(m.q, m.k, m.v, m.bias, p);
     return cudaGetLastError();
@@ -264,7 +333,7 @@ attn_status_t validate_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const
     *empty = false;
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
     // dtype rules first: fp32 is a valid request this fused kernel does not serve
-    if (q->dtype == ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+    if (q->dtype == ATTN_F32 || q->dtype == ATTN_E4M3) return ATTN_ERR_UNSUPPORTED;   // (e4m3: attn_fwd_fp8)
     if (!is_half_type(q->dtype)) return ATTN_ERR_INVALID_ARG;
     if (k->dtype != q->dtype || v->dtype != q->dtype || out->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
     if (bias != nullptr && bias->dtype != q->dtype) return ATTN_ERR_UNSUPPORTED;
@@ -310,33 +379,49 @@ attn_status_t validate_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const
     return ATTN_OK;
 }
 
-// ---------------------------------------------------------------------------
-// backward launches
-// ---------------------------------------------------------------------------
-template <typename T, int D, bool CAUSAL>
-cudaError_t launch_bwd_t(const attn::bwd::BwdParams& p, cudaStream_t stream) {
-    constexpr int smem = attn::bwd::BwdSmem<D>::kBytes;
-    auto kdkdv = attn::bwd::attn_bwd_dkdv_kernel<T, D, CAUSAL>;
-    auto kdq = attn::bwd::attn_bwd_dq_kernel<T, D, CAUSAL>;
-    cudaError_t e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+// Tensor-core backward: D_i into dQ's rows, then dK/dV (one CTA per 128 keys), then dQ (one CTA
+// per 128 queries).  m: Q/dO maps with 64-row boxes and K/V with 128 (dK/dV kernel), then
+// Q/dO with 128 and K/V with 64 (dQ kernel).
+struct BwdMaps {
+    CUtensorMap q64, k128, v128, do64, q128, k64, v64, do128;
+};
+
+template <typename T, int D, bool CAUSAL, bool MODS>
+cudaError_t launch_bwd_tc_t(const BwdMaps& m, const attn::bwdtc::Params& p, cudaStream_t stream) {
+    using namespace attn::bwdtc;
+    const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
+    const int64_t blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+    bwd_prep_kernel<T, D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    const dim3 g_kv((p.Nk + attn::bwd::kRows - 1) / attn::bwd::kRows, p.B * p.H);
-    const dim3 g_q((p.N + attn::bwd::kRows - 1) / attn::bwd::kRows, p.B * p.H);
-    kdkdv<<<g_kv, attn::bwd::kThreads, smem, stream>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    kdq<<<g_q, attn::bwd::kThreads, smem, stream>>>(p);
+    auto k1 = bwd_dkdv_kernel<T, D, CAUSAL, MODS>;
+    constexpr int s1 = DkdvCfg<D>::kDynBytes;
+    static std::atomic<uint64_t> set1{0}, set2{0};
+    if ((e = smem_limit_once(k1, s1, set1)) != cudaSuccess) return e;
+    k1<<<dim3((p.Nk + 127) / 128, p.B * p.H), kThreads, s1, stream>>>(m.q64, m.k128, m.v128, m.do64, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    auto k2 = bwd_dq_kernel<T, D, CAUSAL, MODS>;
+    constexpr int s2 = DqCfg<D>::kDynBytes;
+    if ((e = smem_limit_once(k2, s2, set2)) != cudaSuccess) return e;
+    k2<<<dim3((p.N + 127) / 128, p.B * p.H), kThreads, s2, stream>>>(m.q128, m.k64, m.v64, m.do128, p);
     return cudaGetLastError();
 }
 
-template <typename T>
-cudaError_t launch_bwd_dtype(int d, bool causal, const attn::bwd::BwdParams& p, cudaStream_t s) {
-    if (d == 32) return causal ? launch_bwd_t<T, 32, true>(p, s) : launch_bwd_t<T, 32, false>(p, s);
-    if (d == 64) return causal ? launch_bwd_t<T, 64, true>(p, s) : launch_bwd_t<T, 64, false>(p, s);
-    return causal ? launch_bwd_t<T, 128, true>(p, s) : launch_bwd_t<T, 128, false>(p, s);
+template <typename T, int D>
+cudaError_t launch_bwd_tc_d(bool causal, bool mods, const BwdMaps& m, const attn::bwdtc::Params& p, cudaStream_t s) {
+    if (mods) return causal ? launch_bwd_tc_t<T, D, true, true>(m, p, s) : launch_bwd_tc_t<T, D, false, true>(m, p, s);
+    return causal ? launch_bwd_tc_t<T, D, true, false>(m, p, s) : launch_bwd_tc_t<T, D, false, false>(m, p, s);
 }
+
+template <typename T>
+cudaError_t launch_bwd_tc_dtype(int d, bool causal, bool mods, const BwdMaps& m, const attn::bwdtc::Params& p,
+                                cudaStream_t s) {
+    if (d == 32) return launch_bwd_tc_d<T, 32>(causal, mods, m, p, s);
+    if (d == 64) return launch_bwd_tc_d<T, 64>(causal, mods, m, p, s);
+    return launch_bwd_tc_d<T, 128>(causal, mods, m, p, s);
+}
+
 
 // A host view and its device staging view: same dtype, rank, shape and strides.
 bool same_layout(const attn_tensor_t* a, const attn_tensor_t* b) {
@@ -676,6 +761,19 @@ attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
                        const attn_tensor_t* out, const float* lse, const attn_tensor_t* dout, int causal,
                        float scale, attn_tensor_t* dq, attn_tensor_t* dk, attn_tensor_t* dv,
                        cudaStream_t stream) {
+    return attn_bwd_ex(q, k, v, out, lse, dout, causal, scale, nullptr, dq, dk, dv, stream);
+}
+
+attn_status_t attn_bwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                          const attn_tensor_t* out, const float* lse, const attn_tensor_t* dout, int causal,
+                          float scale, const attn_mods_t* mods, attn_tensor_t* dq, attn_tensor_t* dk,
+                          attn_tensor_t* dv, cudaStream_t stream) {
+    bool mods_on = false;
+    if (mods != nullptr) {
+        if (!std::isfinite(mods->softcap) || mods->softcap < 0.f) return ATTN_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(mods->alibi_slopes) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+        mods_on = mods->alibi_slopes != nullptr || mods->softcap > 0.f || mods->window_left >= 0;
+    }
     bool empty = false;
     attn_status_t st = validate_fwd(q, k, v, nullptr, nullptr, scale, out, lse, &empty);
     if (st != ATTN_OK) return st;
@@ -706,25 +804,35 @@ attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
     }
     if (B * H > 65535) return ATTN_ERR_UNSUPPORTED;
 
-    attn::bwd::BwdParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.B = static_cast<int>(B);
-    p.H = static_cast<int>(H);
-    p.N = static_cast<int>(N);
-    p.Nk = static_cast<int>(Nk);
-    p.causal_off = static_cast<int>(Nk - N);
-    p.scale = scale;
-    p.q = q->data; p.q_sb = q->stride[0]; p.q_sh = q->stride[1]; p.q_si = q->stride[2];
-    p.k = k->data; p.k_sb = k->stride[0]; p.k_sh = k->stride[1]; p.k_si = k->stride[2];
-    p.v = v->data; p.v_sb = v->stride[0]; p.v_sh = v->stride[1]; p.v_si = v->stride[2];
-    p.o = out->data; p.o_sb = out->stride[0]; p.o_sh = out->stride[1]; p.o_si = out->stride[2];
-    p.dout = dout->data; p.do_sb = dout->stride[0]; p.do_sh = dout->stride[1]; p.do_si = dout->stride[2];
-    p.lse = lse;
-    p.dq = dq->data; p.dq_sb = dq->stride[0]; p.dq_sh = dq->stride[1]; p.dq_si = dq->stride[2];
-    p.dk = dk->data; p.dk_sb = dk->stride[0]; p.dk_sh = dk->stride[1]; p.dk_si = dk->stride[2];
-    p.dv = dv->data; p.dv_sb = dv->stride[0]; p.dv_sh = dv->stride[1]; p.dv_si = dv->stride[2];
-    cudaError_t e = q->dtype == ATTN_BF16 ? launch_bwd_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, p, stream)
-                                          : launch_bwd_dtype<__half>(static_cast<int>(d), causal != 0, p, stream);
+    attn::bwdtc::Params tp;
+    std::memset(&tp, 0, sizeof(tp));
+    tp.B = static_cast<int>(B);
+    tp.H = static_cast<int>(H);
+    tp.N = static_cast<int>(N);
+    tp.Nk = static_cast<int>(Nk);
+    tp.causal_off = static_cast<int>(Nk - N);
+    tp.scale = scale;
+    tp.scale_log2 = scale * 1.4426950408889634f;
+    tp.o = out->data; tp.o_sb = out->stride[0]; tp.o_sh = out->stride[1]; tp.o_si = out->stride[2];
+    tp.dout = dout->data; tp.do_sb = dout->stride[0]; tp.do_sh = dout->stride[1]; tp.do_si = dout->stride[2];
+    tp.lse = lse;
+    tp.dq = dq->data; tp.dq_sb = dq->stride[0]; tp.dq_sh = dq->stride[1]; tp.dq_si = dq->stride[2];
+    tp.dk = dk->data; tp.dk_sb = dk->stride[0]; tp.dk_sh = dk->stride[1]; tp.dk_si = dk->stride[2];
+    tp.dv = dv->data; tp.dv_sb = dv->stride[0]; tp.dv_sh = dv->stride[1]; tp.dv_si = dv->stride[2];
+    tp.wait_limit = g_wait_limit;
+    tp.status = status_word_ptr();
+    tp.alibi = mods_on ? mods->alibi_slopes : nullptr;
+    tp.softcap = mods_on ? mods->softcap : 0.f;
+    tp.window_left = (mods_on && mods->window_left >= 0) ? mods->window_left : -1;
+    if (tp.status == nullptr) return ATTN_ERR_CUDA;
+    BwdMaps m;
+    if (!encode_qkv_map(&m.q64, q, 64) || !encode_qkv_map(&m.k128, k, 128) || !encode_qkv_map(&m.v128, v, 128) ||
+        !encode_qkv_map(&m.do64, dout, 64) || !encode_qkv_map(&m.q128, q, 128) || !encode_qkv_map(&m.k64, k, 64) ||
+        !encode_qkv_map(&m.v64, v, 64) || !encode_qkv_map(&m.do128, dout, 128))
+        return ATTN_ERR_CUDA;
+    cudaError_t e = q->dtype == ATTN_BF16
+                        ? launch_bwd_tc_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, mods_on, m, tp, stream)
+                        : launch_bwd_tc_dtype<__half>(static_cast<int>(d), causal != 0, mods_on, m, tp, stream);
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -755,5 +863,114 @@ void attn_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles < 1024 ? 1024 
 void attn_debug_inject_stall(int enable) { g_inject_stall = enable != 0; }
 
 const char* attn_version(void) { return "0.1.0"; }
+
+}  // extern "C"
+
+namespace {
+// e4m3 tensor: positive shape, unit inner stride, other strides multiples of 16 elements (bytes),
+// 16-byte aligned data
+attn_status_t check_e4m3(const attn_tensor_t* t) {
+    if (t == nullptr || t->data == nullptr || t->dtype != ATTN_E4M3 || t->ndim != 4) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i)
+        if (t->shape[i] <= 0) return ATTN_ERR_INVALID_ARG;
+    if (t->stride[3] != 1) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i) {
+        if (t->stride[i] < 0 || (t->stride[i] % 16) != 0) return ATTN_ERR_INVALID_ARG;
+        if (t->shape[i] > 1 && t->stride[i] == 0) return ATTN_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(t->data) & 15u) != 0) return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+
+int64_t span_bytes_e(const attn_tensor_t* t, int64_t esize) {
+    int64_t last = 0;
+    for (int i = 0; i < t->ndim; ++i) last += (t->shape[i] - 1) * t->stride[i];
+    return (last + 1) * esize;
+}
+
+bool overlaps_e(const attn_tensor_t* a, int64_t ea, const attn_tensor_t* b, int64_t eb) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a->data), a1 = a0 + span_bytes_e(a, ea);
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(b->data), b1 = b0 + span_bytes_e(b, eb);
+    return a0 < b1 && b0 < a1;
+}
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd_fp8(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v_t, float q_scale,
+                           float k_scale, float v_scale, int causal, float scale, attn_tensor_t* out, float* lse,
+                           cudaStream_t stream) {
+    if (q == nullptr || k == nullptr || v_t == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (q->dtype != ATTN_E4M3 || k->dtype != ATTN_E4M3 || v_t->dtype != ATTN_E4M3) return ATTN_ERR_UNSUPPORTED;
+    if (!is_half_type(out->dtype)) return ATTN_ERR_UNSUPPORTED;
+    for (float f : {q_scale, k_scale, v_scale, scale})
+        if (!std::isfinite(f)) return ATTN_ERR_INVALID_ARG;
+    if (q_scale <= 0.f || k_scale <= 0.f || v_scale <= 0.f) return ATTN_ERR_INVALID_ARG;
+    attn_status_t st;
+    if ((st = check_e4m3(q)) != ATTN_OK || (st = check_e4m3(k)) != ATTN_OK || (st = check_e4m3(v_t)) != ATTN_OK)
+        return st;
+    if ((st = check_tensor(out, 4)) != ATTN_OK) return st;
+    if (!same_shape(q, out) || !same_bhd(q, k)) return ATTN_ERR_INVALID_ARG;
+    // V transposed: [B, H, d, Nk]
+    if (v_t->shape[0] != k->shape[0] || v_t->shape[1] != k->shape[1] || v_t->shape[2] != k->shape[3] ||
+        v_t->shape[3] != k->shape[2])
+        return ATTN_ERR_INVALID_ARG;
+    const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (N > (int64_t(1) << 30) || Nk > (int64_t(1) << 30) || B * H > (int64_t(1) << 24)) return ATTN_ERR_UNSUPPORTED;
+    if (overlaps_e(out, 2, q, 1) || overlaps_e(out, 2, k, 1) || overlaps_e(out, 2, v_t, 1)) return ATTN_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+
+    Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!encode_e4m3_map(&maps.q, q) || !encode_e4m3_map(&maps.k, k) || !encode_e4m3_vt_map(&maps.v, v_t))
+        return ATTN_ERR_CUDA;
+    unsigned int* status = status_word_ptr();
+    if (status == nullptr) return ATTN_ERR_CUDA;
+    FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = static_cast<int>(B);
+    p.H = static_cast<int>(H);
+    p.N = static_cast<int>(N);
+    p.Nk = static_cast<int>(Nk);
+    p.causal_off = static_cast<int>(Nk - N);
+    p.num_q_pairs = static_cast<int>((N + attn::kRowsPerUnit - 1) / attn::kRowsPerUnit);
+    p.n_kv_tiles = static_cast<int>((Nk + attn::kBlockN - 1) / attn::kBlockN);
+    const int64_t units = static_cast<int64_t>(p.num_q_pairs) * B * H;
+    if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    p.num_units = static_cast<int>(units);
+    // the query and key scales fold into the score scale; the value scale into the epilogue
+    const double s_all = static_cast<double>(scale) * q_scale * k_scale;
+    p.scale = static_cast<float>(s_all);
+    p.scale_log2 = static_cast<float>(s_all * 1.4426950408889634);
+    p.v_scale = v_scale;
+    {
+        const double kv_bytes = 2.0 * static_cast<double>(B * H) * static_cast<double>(Nk) * d;
+        const int sms = sm_count();
+        int g = static_cast<int>(B * H);
+        if (sms > 0 && kv_bytes > static_cast<double>(l2_bytes())) g = (sms + p.num_q_pairs - 1) / p.num_q_pairs;
+        p.head_group = g < 1 ? 1 : (g > B * H ? static_cast<int>(B * H) : g);
+    }
+    p.out = out->data;
+    p.out_sb = out->stride[0];
+    p.out_sh = out->stride[1];
+    p.out_si = out->stride[2];
+    p.lse = lse;
+    p.lse_sh = N;
+    p.lse_sb = H * N;
+    p.window_left = -1;
+    p.wait_limit = g_wait_limit;
+    p.status = status;
+    p.inject_stall = g_inject_stall;
+    cudaError_t e;
+    const bool bf = out->dtype == ATTN_BF16;
+    if (d == 64)
+        e = bf ? (causal ? launch_fp8_t<__nv_bfloat16, 64, true>(maps, p, stream) : launch_fp8_t<__nv_bfloat16, 64, false>(maps, p, stream))
+               : (causal ? launch_fp8_t<__half, 64, true>(maps, p, stream) : launch_fp8_t<__half, 64, false>(maps, p, stream));
+    else
+        e = bf ? (causal ? launch_fp8_t<__nv_bfloat16, 128, true>(maps, p, stream) : launch_fp8_t<__nv_bfloat16, 128, false>(maps, p, stream))
+               : (causal ? launch_fp8_t<__half, 128, true>(maps, p, stream) : launch_fp8_t<__half, 128, false>(maps, p, stream));
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 }  // extern "C"

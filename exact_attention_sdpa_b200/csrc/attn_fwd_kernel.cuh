@@ -91,6 +91,7 @@ struct FwdParams {
     unsigned long long wait_limit;
     unsigned int* status;
     int inject_stall;          // test hook: the MMA warp first waits on a barrier nothing arrives on
+    float v_scale;             // e4m3 inputs: the value tensor's scale (the query and key scales are in scale)
     // ragged batch in one launch (n_seq > 0; B = 1 and the tensors are packed [1, H, T, d] views):
     // sequence s owns query rows seq_q0[s] .. + seq_nq[s] and key rows seq_k0[s] .. + seq_nk[s],
     // and units seq_units[s] .. seq_units[s + 1] (its query pairs x H, heaviest pairs first)
@@ -99,18 +100,29 @@ struct FwdParams {
     int seq_q0[kMaxSeq], seq_k0[kMaxSeq], seq_nq[kMaxSeq], seq_nk[kMaxSeq];
 };
 
-template <int D>
+template <int D, bool FP8 = false>
 struct Cfg {
     static_assert(D == 32 || D == 64 || D == 128, "head dim");
+    static_assert(!FP8 || D >= 64, "e4m3 inputs: d = 64 or 128");
     // A 128-row tile of D 16-bit elements is stored as D/64 "atoms" of 128 rows
     // x 128 bytes (128-byte swizzle), or for D = 32 one atom of 128 rows x 64
-    // bytes (64-byte swizzle): exactly the layout TMA writes.
-    static constexpr int kAtomCols = (D >= 64) ? 64 : 32;
+    // bytes (64-byte swizzle): exactly the layout TMA writes.  With e4m3 inputs a
+    // row of D bytes is one atom: 64 bytes (64-byte swizzle) or 128 bytes (128-byte).
+    static constexpr int kElemBytes = FP8 ? 1 : 2;
+    static constexpr int kRowBytes = FP8 ? D : ((D >= 64) ? 128 : 64);
+    static constexpr int kAtomCols = kRowBytes / kElemBytes;
     static constexpr int kNumAtoms = D / kAtomCols;
-    static constexpr int kRowBytes = kAtomCols * 2;
     static constexpr int kAtomBytes = 128 * kRowBytes;
-    static constexpr int kTileBytes = kNumAtoms * kAtomBytes;     // 128 * D * 2
-    static constexpr uint32_t kLayout = (D >= 64) ? 2u : 4u;      // SW128 : SW64
+    static constexpr int kTileBytes = kNumAtoms * kAtomBytes;     // 128 * D * element bytes
+    static constexpr uint32_t kLayout = (kRowBytes == 128) ? 2u : 4u;   // SW128 : SW64
+    // reduction elements per MMA instruction: always 32 bytes (16 halves or 32 e4m3 values)
+    static constexpr int kK = 32 / kElemBytes;
+    // offset (16-byte units) of the kk-th reduction step in a K-major tile
+    static __host__ __device__ constexpr uint32_t kstep(int kk) {
+        return static_cast<uint32_t>((((kk * 32) / kRowBytes) * kAtomBytes + (kk * 32) % kRowBytes) >> 4);
+    }
+    // tensor-memory columns of one tile's P: 128 keys packed into 32-bit columns
+    static constexpr uint32_t kColsP = 128 * kElemBytes / 4;
     static constexpr uint32_t kSBO = 8 * kRowBytes;               // 8-row group stride
     static constexpr int kStages = (D == 128) ? 2 : (D == 64 ? 3 : 4);
     // tensor memory columns
@@ -123,8 +135,8 @@ struct Cfg {
     static constexpr int kEmuPeriod = (D == 64) ? 4 : 0;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColP0 = (D == 128) ? 0 : 256;
-    static constexpr uint32_t kColP1 = (D == 128) ? 128 : 320;
-    static constexpr uint32_t kColO0 = (D == 128) ? 256 : 384;
+    static constexpr uint32_t kColP1 = (D == 128) ? 128 : 256 + kColsP;
+    static constexpr uint32_t kColO0 = (D == 128) ? 256 : 256 + 2 * kColsP;
     static constexpr uint32_t kColO1 = kColO0 + ((D == 128) ? 128 : D);
     static_assert(kColO1 + D <= kTmemCols, "tensor memory budget");
     // shared memory (dynamic, 1024-byte aligned)
@@ -338,15 +350,18 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
 }
 
 // MODS: score modifications compiled in (only without bias and gate); other builds carry none of it.
-template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE, bool MODS = false>
+// FP8: Q, K and V (transposed) are e4m3 codes and T is the output type; the plain path only.
+template <typename T, int D, bool CAUSAL, bool HAS_BIAS, bool HAS_GATE, bool MODS = false, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
                     const __grid_constant__ FwdParams p) {
     using namespace sm100;
-    using C = Cfg<D>;
+    using C = Cfg<D, FP8>;
+    static_assert(!FP8 || (!HAS_BIAS && !HAS_GATE && !MODS), "e4m3 inputs: plain path only");
     constexpr int ST = C::kStages;
-    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    // operand format bits of the instruction descriptor: 1 selects bf16 (kind::f16); e4m3 is 0
+    constexpr bool kBF16 = !FP8 && std::is_same<T, __nv_bfloat16>::value;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ FwdShared<ST> sh;
@@ -401,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* abort_flag = &sh.abort_flag;
 
     if (wg == 3) {
-        regs_dec<Cfg<D>::kRegsOther>();
+        regs_dec<C::kRegsOther>();
         if (warp == 13) {
             // ============================================================ TMA producer
             // The whole warp runs this loop (uniform control flow); one elected lane issues.
@@ -452,11 +467,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                int j, const Unit& U) {
                 const uint32_t st = cnt % ST;
                 if (cnt >= ST && !WU(&empty[st], ((cnt / ST) - 1) & 1)) return;
+                const int key0 = U.k_base + (U.kv_lo + j) * kBlockN;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&full[st], C::kTileBytes);
-                    for (int a = 0; a < C::kNumAtoms; ++a)
-                        tma_load_4d(ring + (st * C::kNumAtoms + a) * C::kAtomBytes, map, &full[st],
-                                    a * C::kAtomCols, U.k_base + (U.kv_lo + j) * kBlockN, U.h, U.b, pol_kv);
+                    if (FP8 && ring == sV) {
+                        // e4m3: V arrives transposed ([B, H, d, Nk]); one box of 128 keys x d rows,
+                        // one 128-byte swizzle atom per row, which the PV MMA reads K-major
+                        tma_load_4d(ring + st * C::kTileBytes, map, &full[st], key0, 0, U.h, U.b, pol_kv);
+                    } else {
+                        for (int a = 0; a < C::kNumAtoms; ++a)
+                            tma_load_4d(ring + (st * C::kNumAtoms + a) * C::kAtomBytes, map, &full[st],
+                                        a * C::kAtomCols, key0, U.h, U.b, pol_kv);
+                    }
                 }
                 __syncwarp();
                 ++cnt;
@@ -496,7 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == 12) {
             // ============================================================ MMA issuer
             constexpr uint32_t idesc_s = instr_desc_f16(kBF16, kBlockM, kBlockN, false);
-            constexpr uint32_t idesc_o = instr_desc_f16(kBF16, kBlockM, D, true);
+            // (e4m3: V^T is K-major, like K in S; 16-bit V is N-major)
+            constexpr uint32_t idesc_o = instr_desc_f16(kBF16, kBlockM, D, !FP8);
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t k_addr = smem_u32(sK);
             const uint32_t v_addr = smem_u32(sV);
@@ -507,29 +530,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             // shared addresses stay below 256 KB), so each step adds a constant to a base.
             const uint64_t dq = smem_desc(q_addr, 16, C::kSBO, C::kLayout);
             const uint64_t dk = smem_desc(k_addr, 16, C::kSBO, C::kLayout);
-            const uint64_t dv = smem_desc(v_addr, C::kAtomBytes, C::kSBO, C::kLayout);
-            // S_i = Q_i K^T: both operands K-major, 16 elements (32 bytes) per step
+            // e4m3 V^T: rows of 128 keys (128 bytes, 128-byte swizzle), K-major
+            const uint64_t dv = FP8 ? smem_desc(v_addr, 16, 8 * 128, 2u)
+                                    : smem_desc(v_addr, C::kAtomBytes, C::kSBO, C::kLayout);
+            // S_i = Q_i K^T: both operands K-major, 32 bytes of the head dim per step
             auto issue_s = [&](int i, uint32_t kst) {
                 const uint64_t qb = dq + ((i * C::kTileBytes) >> 4);
                 const uint64_t kb = dk + ((kst * C::kTileBytes) >> 4);
                 if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off =
-                            (((kk * 16) / C::kAtomCols) * C::kAtomBytes + ((kk * 16) % C::kAtomCols) * 2) >> 4;
-                        mma_ss(tmem + kColS[i], qb + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / C::kK; ++kk) {
+                        const uint32_t off = C::kstep(kk);
+                        if constexpr (FP8) mma_ss_f8(tmem + kColS[i], qb + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
+                        else mma_ss(tmem + kColS[i], qb + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
                     }
                 }
                 __syncwarp();
             };
-            // O_i += P_i V: P from tensor memory, V N(=d)-major in shared memory, 16 keys per step
+            // O_i += P_i V: P from tensor memory (8 columns per step), kK keys per step of V: kK rows
+            // of the N(=d)-major 16-bit V, or 32 bytes along each row of the e4m3 V^T
             auto issue_pv = [&](int i, uint32_t vst, bool acc) {
                 const uint64_t vb = dv + ((vst * C::kTileBytes) >> 4);
                 if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk)
-                        mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8, vb + ((kk * 16 * C::kRowBytes) >> 4),
-                               idesc_o, (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBlockN / C::kK; ++kk) {
+                        const uint64_t vk = vb + (FP8 ? ((kk * 32) >> 4) : ((kk * C::kK * C::kRowBytes) >> 4));
+                        if constexpr (FP8)
+                            mma_ts_f8(tmem + kColO[i], tmem + kColP[i] + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
+                        else
+                            mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
+                    }
                 }
                 __syncwarp();
             };
@@ -672,12 +702,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (wg < 2) {
         // ================================================================ softmax of tile i = wg
-        regs_inc<Cfg<D>::kRegsSoftmax>();
+        regs_inc<C::kRegsSoftmax>();
         const int i = wg;
         const int t = threadIdx.x & 127;          // row within the tile
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t col_s = i ? Cfg<D>::kColS1 : Cfg<D>::kColS0;
-        const uint32_t col_p = i ? Cfg<D>::kColP1 : Cfg<D>::kColP0;
+        const uint32_t col_s = i ? C::kColS1 : C::kColS0;
+        const uint32_t col_p = i ? C::kColP1 : C::kColP0;
         const float scale_log2 = p.scale_log2;
         const bool fast = !HAS_BIAS && !MODS && scale_log2 > 0.f;   // max over raw scores, fused scale
         uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
@@ -709,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(r[c]);
                 }
-                if constexpr (Cfg<D>::kSeparateP) {
+                if constexpr (C::kSeparateP) {
                     // S_i may now be overwritten by S_i(j+1) (S_i(0) of the next unit is issued
                     // only after this unit's last PV_i, which needs this softmax to finish)
                     if (j + 1 < nkv) {
@@ -810,7 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_new = m_tile;
                     alpha = ex2_approx(m_ref - m_new);
                 }
-                if (!Cfg<D>::kSeparateP && j > 0) {
+                if (!C::kSeparateP && j > 0) {
                     // S_i(j) was issued after PV_i(j-1), so the correction has consumed alpha(j-1)
                     sh.alpha[j & 1][i][t] = alpha;
                     mbar_arrive(&sh.sm2corr[i]);
@@ -825,12 +855,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
+                    float ep0 = 0.f, ep1 = 0.f;     // e4m3: the even pair of the current 32-bit column
 #pragma unroll
                     for (int q2 = 0; q2 < 32; ++q2) {
                         const int pp = half * 32 + q2;
                         float x0, x1, e0, e1;
                         ffma2(x0, x1, s[2 * pp], s[2 * pp + 1], xa, xa, xb, xb);
-                        constexpr int kEmu = Cfg<D>::kEmuPeriod;
+                        constexpr int kEmu = C::kEmuPeriod;
                         if (kEmu > 0 && pp % (kEmu > 0 ? kEmu : 1) == kEmu - 1) {
                             ex2_emu2(e0, e1, x0, x1);
                         } else {
@@ -839,9 +870,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         const int q = (pp & 3) * 2;
                         fadd2_ftz(acc[q], acc[q + 1], acc[q], acc[q + 1], e0, e1);
-                        pk[q2] = pack2<T>(e0, e1);
+                        if constexpr (FP8) {
+                            // four keys per 32-bit column: the even pair waits for the odd one
+                            if (q2 & 1) pk[q2 >> 1] = pack4_e4m3(ep0, ep1, e0, e1);
+                            else { ep0 = e0; ep1 = e1; }
+                        } else {
+                            pk[q2] = pack2<T>(e0, e1);
+                        }
                     }
-                    if constexpr (Cfg<D>::kSeparateP) {
+                    if constexpr (C::kSeparateP) {
                         // P_i(j) overwrites P_i(j-1): PV_i(j-1) must have completed.  Its
                         // completion also means the correction consumed alpha(j-1), so alpha(j)
                         // is published only now (its barrier never runs two phases ahead).
@@ -858,7 +895,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mbar_arrive(&sh.sm2corr[i]);
                         }
                     }
-                    if (ok) tmem_st32(tmem + lane_off + col_p + half * 32, pk);
+                    if constexpr (FP8) {
+                        if (ok) tmem_st16(tmem + lane_off + col_p + half * 16, *reinterpret_cast<uint32_t(*)[16]>(pk));
+                    } else {
+                        if (ok) tmem_st32(tmem + lane_off + col_p + half * 32, pk);
+                    }
                 }
                 tmem_wait_st();
                 if (!ok) break;
@@ -872,7 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The correction must have consumed the previous unit's statistics before this
             // unit's are published: a unit with a single key tile can otherwise finish before
             // the correction reaches the previous epilogue, running stats_full two phases ahead.
-            if constexpr (Cfg<D>::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
+            if constexpr (C::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
             if (uit > 0) {
                 ok = wait_phase(&sh.o_free[i], (uit - 1) & 1, abort_flag, p.wait_limit, p.status);
                 ok = __all_sync(0xffffffffu, ok);
@@ -884,10 +925,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================================ correction + epilogue
-        regs_dec<Cfg<D>::kRegsCorrection>();
+        regs_dec<C::kRegsCorrection>();
         const int t = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        constexpr uint32_t kColO[2] = {Cfg<D>::kColO0, Cfg<D>::kColO1};
+        constexpr uint32_t kColO[2] = {C::kColO0, C::kColO1};
         uint32_t c_cnt[2] = {0, 0}, st_cnt[2] = {0, 0}, od_cnt[2] = {0, 0}, uit = 0;
         bool ok = true;
         auto WS = [&](uint64_t* bar, uint32_t& cnt) {
@@ -958,7 +999,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const float m = sh.stat_m[uit & 1][i][t];
                 const float l = sh.stat_l[uit & 1][i][t];
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                // (e4m3 inputs: the value tensor's scale comes in here)
+                const float inv_l = (l > 0.f) ? (FP8 ? p.v_scale / l : 1.f / l) : 0.f;
                 // one 32-column chunk of O: normalise, gate, round, store
                 auto finish_chunk = [&](const uint32_t (&r)[32], int c) {
                     if (!row_ok) return;

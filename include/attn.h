@@ -45,7 +45,8 @@ typedef enum {
 typedef enum {
     ATTN_F16 = 0,
     ATTN_BF16 = 1,
-    ATTN_F32 = 2                /* accepted by the type only so that it can be rejected (UNSUPPORTED) */
+    ATTN_F32 = 2,               /* accepted by the type only so that it can be rejected (UNSUPPORTED) */
+    ATTN_E4M3 = 3               /* 8-bit float e4m3, finite variant (max 448): attn_fwd_fp8 inputs only */
 } attn_dtype_t;
 
 /*
@@ -214,8 +215,10 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
  * Layout rules and errors as attn_fwd; additionally ATTN_ERR_INVALID_ARG for a
  * missing lse, dout, dq, dk or dv, a shape mismatch or an overlap (lse's
  * B*H*N floats included: they must not overlap dq, dk or dv), and
- * ATTN_ERR_UNSUPPORTED for B*H > 65535.  Asynchronous on `stream` (two kernel
- * launches); allocates nothing.
+ * ATTN_ERR_UNSUPPORTED for B*H > 65535.  Asynchronous on `stream`, three kernel
+ * launches on the tensor cores: D_i (written as an fp32 into the first bytes of
+ * dq's row i, which the last launch then overwrites with dQ), dK/dV (one CTA per
+ * 128 keys), dQ (one CTA per 128 queries); no atomics, allocates nothing.
  */
 attn_status_t attn_bwd(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                        const attn_tensor_t* out, const float* lse, const attn_tensor_t* dout, int causal,
@@ -262,6 +265,43 @@ void attn_set_wait_limit(uint64_t cycles);
 void attn_debug_inject_stall(int enable);
 
 /*
+ * attn_fwd_fp8 -- the forward on 8-bit (e4m3) inputs with per-tensor scales: the
+ * low-precision variant of hamidun.com's FlashAttention-3 article (the FP8
+ * section: about twice the 16-bit throughput, error close to plain FP8
+ * attention).  The page fixes no format or scaling rule; the readings taken:
+ *
+ *   element x of q, k or v_t stands for decode_e4m3(x) * that tensor's scale;
+ *   O and lse are those of attn_fwd's exact operation on those values; the
+ *   kernel's one added rounding is P's: each p (relative to the running row
+ *   maximum, at most 2^8) is rounded to e4m3 (nearest even, saturating) before
+ *   P V runs on the 8-bit tensor core, while the row sum l adds the unrounded p.
+ *   Per output element the result then differs from the exact one by at most
+ *   sum_j max(2^-4 p_ij, 2^-10) |v_jc| / l_i (p against the row maximum), plus
+ *   out's own rounding.
+ *
+ *   q        [B, H, N, d]  e4m3 codes (ATTN_E4M3), device memory; d in {64, 128}.
+ *   k        [B, H, Nk, d] e4m3.
+ *   v_t      V TRANSPOSED: [B, H, d, Nk] e4m3 (both tensor-core operands of P V are
+ *            then read along the key axis).
+ *   q_scale, k_scale, v_scale   finite, > 0.
+ *   causal, scale               as attn_fwd (scale multiplies the decoded, scaled
+ *                               Q K^T; q_scale * k_scale * scale is folded into one
+ *                               factor, v_scale into the epilogue).
+ *   out      [B, H, N, d] fp16 or bf16 (the output type).
+ *   lse      nullable; [B, H, N] fp32 as attn_fwd.
+ *
+ * Layout: inner stride 1; every other stride a multiple of 16 elements (bytes for
+ * the e4m3 tensors); 16-byte aligned data.  No bias, gate or score modification.
+ * ATTN_ERR_UNSUPPORTED for non-e4m3 inputs, another d or an out dtype other than
+ * fp16/bf16; ATTN_ERR_INVALID_ARG for nulls, shape mismatches, a non-finite or
+ * non-positive scale, misalignment, or out overlapping an input.  Asynchronous on
+ * `stream`; allocates nothing.
+ */
+attn_status_t attn_fwd_fp8(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v_t, float q_scale,
+                           float k_scale, float v_scale, int causal, float scale, attn_tensor_t* out, float* lse,
+                           cudaStream_t stream);
+
+/*
  * attn_debug_exp2 -- test hook: evaluates, on the device, one of the base-2
  * exponentials the forward kernel's softmax uses, so that each can be checked
  * against the exact value and against CUDA's exp2f.  Not part of the
@@ -285,6 +325,17 @@ attn_status_t attn_debug_exp2(const float* x, float* y, int64_t n, int mode, cud
 
 /* The library version as "major.minor.patch" (static string). */
 const char* attn_version(void);
+
+
+/*
+ * attn_bwd_ex -- attn_bwd for a forward run with score modifications (`mods` as given to
+ * attn_fwd_ex; nullable: none).  The softcap's derivative 1 - tanh(s / c)^2 enters dS; the ALiBi
+ * shift and the window mask only change P.  Errors as attn_bwd, plus those of attn_fwd_ex's mods.
+ */
+attn_status_t attn_bwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                          const attn_tensor_t* out, const float* lse, const attn_tensor_t* dout, int causal,
+                          float scale, const attn_mods_t* mods, attn_tensor_t* dq, attn_tensor_t* dk,
+                          attn_tensor_t* dv, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -378,3 +378,25 @@ def test_plain_c_client_compiles_links_and_calls(lib, tmp_path):
     assert r.returncode == 0, r.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
+
+
+def test_fp8_argument_checks(lib):
+    """attn_fwd_fp8 rejects what it does not serve before any launch."""
+    f8 = lambda *shape: torch.zeros(*shape, dtype=torch.uint8).view(torch.float8_e4m3fn)
+    q, k = f8(1, 2, 64, 64), f8(1, 2, 80, 64)
+    vt = f8(1, 2, 64, 80)
+    o = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    call = lambda q_=q, k_=k, v_=vt, o_=o, sq=1.0, sk=1.0, sv=1.0: nat.attn_fwd_fp8_raw(
+        q_, k_, v_, sq, sk, sv, True, 0.125, o_, None, 0)
+    assert call(q_=torch.zeros(1, 2, 64, 64, dtype=torch.float16)) == nat.ATTN_ERR_UNSUPPORTED   # not e4m3
+    assert call(o_=torch.zeros(1, 2, 64, 64, dtype=torch.float32)) == nat.ATTN_ERR_UNSUPPORTED   # out fp32
+    assert call(q_=f8(1, 2, 64, 32), k_=f8(1, 2, 80, 32), v_=f8(1, 2, 32, 80),
+                o_=torch.zeros(1, 2, 64, 32, dtype=torch.bfloat16)) == nat.ATTN_ERR_UNSUPPORTED  # d = 32
+    assert call(sq=0.0) == nat.ATTN_ERR_INVALID_ARG
+    assert call(sv=float("nan")) == nat.ATTN_ERR_INVALID_ARG
+    assert call(v_=f8(1, 2, 80, 64)) == nat.ATTN_ERR_INVALID_ARG          # V not transposed
+    assert call(o_=torch.zeros(1, 2, 48, 64, dtype=torch.bfloat16)) == nat.ATTN_ERR_INVALID_ARG
+    bad = f8(1, 2, 64, 72)[..., :64]                                     # row stride 72 bytes: not 16-aligned
+    assert call(q_=bad) == nat.ATTN_ERR_INVALID_ARG
+    # e4m3 given to the 16-bit entry point
+    assert nat.attn_fwd_raw(q, q, q, None, None, False, 0.1, o, None, 0) == nat.ATTN_ERR_UNSUPPORTED

@@ -64,3 +64,53 @@ def test_backward_deterministic():
     for _ in range(3):
         again = attn_bwd(q, k, v, out, lse, do, causal=True, scale=w.scale)
         assert all(torch.equal(a, b) for a, b in zip(first, again))
+
+
+MOD_CASES = [  # N, Nk, d, causal, dtype, softcap, alibi, window
+    (300, 300, 64, True, "fp16", 2.0, False, -1),
+    (257, 400, 128, True, "bf16", 0.0, True, -1),
+    (400, 400, 32, True, "bf16", 0.0, False, 100),
+    (300, 700, 64, True, "bf16", 1.5, True, 200),
+    (200, 200, 64, False, "fp16", 3.0, True, 50),
+]
+
+
+@pytest.mark.parametrize("N,Nk,d,causal,dtype,softcap,alibi,window", MOD_CASES)
+def test_backward_with_score_modifications(N, Nk, d, causal, dtype, softcap, alibi, window):
+    H = 3
+    w = Workload("bwdm", B=2, H=H, N=N, d=d, dtype=dtype, causal=causal, seed=150 + N % 11, Nk=Nk)
+    inp = make_inputs(w)
+    do = make_grad_output(w)
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32) if alibi else None
+    dev = torch.device("cuda")
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    sd = None if slopes is None else slopes.to(dev)
+    out, lse = attn_fwd(q, k, v, causal=causal, scale=w.scale, softcap=softcap, alibi_slopes=sd, window_left=window)
+    dq, dk, dv = attn_bwd(q, k, v, out, lse, do.to(dev), causal=causal, scale=w.scale, softcap=softcap,
+                          alibi_slopes=sd, window_left=window)
+    torch.cuda.synchronize()
+    assert last_device_status() == 0
+    rq, rk, rv = sdpa_backward(inp["q"], inp["k"], inp["v"], do, causal=causal, scale=w.scale, softcap=softcap,
+                               alibi_slopes=slopes, window_left=window)
+    for g, r, name in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        _check(g, r, w.torch_dtype, f"{name} mods N={N} Nk={Nk} d={d}")
+
+
+def test_backward_full_size_two_heads():
+    """The N=8192 causal fp16 workload in the launch configuration the benchmark times; the
+    oracle's gradients of two whole (b, h) heads are compared element by element."""
+    from exact_attention_sdpa_b200.workloads import WORKLOADS
+    w = WORKLOADS["n8192_causal"]
+    inp = make_inputs(w)
+    do = make_grad_output(w)
+    dev = torch.device("cuda")
+    q, k, v = (inp[n].to(dev) for n in "qkv")
+    out, lse = attn_fwd(q, k, v, causal=True, scale=w.scale)
+    dq, dk, dv = attn_bwd(q, k, v, out, lse, do.to(dev), causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert last_device_status() == 0
+    for b, h in ((0, 0), (w.B - 1, w.H - 1)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        rq, rk, rv = sdpa_backward(inp["q"][sl], inp["k"][sl], inp["v"][sl], do[sl], causal=True, scale=w.scale)
+        for g, r, name in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+            _check(g[sl], r, w.torch_dtype, f"{name} n8192 head ({b},{h})")
