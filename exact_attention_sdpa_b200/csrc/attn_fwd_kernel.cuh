@@ -25,13 +25,14 @@
 // Warp roles (16 warps):
 //   WG0 (warps 0-3)   softmax of Q0: thread t owns query row t; reads its score
 //                     row from tensor memory, masks/scales, updates m and l,
-//                     writes P (fp16/bf16) back to tensor memory.
+//                     writes P (fp16/bf16) back to tensor memory.  When m grew by
+//                     more than 2^8 the O accumulator row is rescaled (otherwise
+//                     the stale maximum is kept: the final O/l and lse use the
+//                     same reference, so the result is unchanged): at d <= 64 by
+//                     the softmax thread itself, at d = 128 by WG2.
 //   WG1 (warps 4-7)   the same for Q1.
-//   WG2 (warps 8-11)  correction: rescales the O accumulators in tensor memory
-//                     when m grew by more than 2^8 (otherwise the stale maximum
-//                     is kept: the final O/l and lse use the same reference, so
-//                     the result is unchanged), then the epilogue: O/l, gate,
-//                     rounding, stores of O and lse.
+//   WG2 (warps 8-11)  epilogue: O/l, gate, rounding, stores of O and lse; at
+//                     d = 128 also the correction (the O rescale above).
 //   warp 12           tcgen05.mma issuer (one thread); allocates tensor memory.
 //   warp 13           TMA producer: Q0, Q1 per unit, K and V tiles into rings.
 //   warps 14-15       idle (they complete warpgroup 3's register hand-back).
@@ -129,6 +130,14 @@ struct Cfg {
     // d <= 64: P has columns of its own, so S_i(j+1) may be computed while the
     // softmax of S_i(j) runs; d = 128: P lives inside S_i (no room otherwise).
     static constexpr bool kSeparateP = (D <= 64);
+    // Who rescales O when a row maximum moves.  With separate P columns the softmax warps do it
+    // themselves, after waiting for the previous PV (which they wait for anyway before P is
+    // overwritten), so PV_i(j) waits only for the softmax.  At d = 128 (P inside S) the softmax
+    // has no such wait and no registers to spare: the correction warpgroup rescales O between
+    // PV_i(j-1) and PV_i(j) and PV_i(j) waits for both (measured on B200: each choice is the
+    // faster one for its head dim).
+    static constexpr bool kInlineRescale = kSeparateP;
+    static constexpr uint32_t kPvArrivals = kInlineRescale ? kBlockM : 2 * kBlockM;
     // One exponential pair in kEmuPeriod goes through the FMA-pipe 2^x (0: none).  Measured
     // on B200: at d=64 one in four beats one in three and none; at d=128 (MMA-bound) and
     // d=32 (short units) the extra FMA-pipe work costs more than the MUFU time it saves.
@@ -146,14 +155,14 @@ struct Cfg {
     static constexpr int kBytes = kOffV + kStages * kTileBytes;
     static constexpr int kDynBytes = kBytes + 1024;
     static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
-    // per-thread registers after setmaxnreg: 256 softmax + 128 correction + 128 other
+    // per-thread registers after setmaxnreg: 256 softmax + 128 epilogue + 128 other
     // threads must fit the 65536 the CTA was launched with (512 threads x 128)
-    // (d=64: the MMA issuer and TMA producer get 96, the correction 64 - fewer spills in the
+    // (d=64: the MMA issuer and TMA producer get 96, the epilogue 64 - fewer spills in the
     // issuer's loop, measured 2-3 % faster than 80 / 80 at N=8192)
     static constexpr int kRegsSoftmax = 176;
-    static constexpr int kRegsCorrection = (D == 64) ? 64 : 80;
+    static constexpr int kRegsEpilogue = (D == 64) ? 64 : 80;
     static constexpr int kRegsOther = (D == 64) ? 96 : 80;
-    static_assert(256 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= 65536, "register budget");
+    static_assert(256 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= 65536, "register budget");
 };
 
 // Additive bias staged through shared memory by TMA (d <= 64; at d = 128 the K/V rings
@@ -179,17 +188,18 @@ struct __align__(8) FwdShared {
     uint64_t k_full[ST], k_empty[ST], v_full[ST], v_empty[ST];
     uint64_t s_full[2];      // MMA -> softmax i: S_i(j) in tensor memory
     uint64_t s_free[2];      // softmax i -> MMA: S_i(j) read into registers (d <= 64 only)
-    uint64_t pv_ready[2];    // softmax i (P written) + correction (O rescaled) -> MMA
-    uint64_t o_done[2];      // MMA -> correction: PV_i(j) complete
-    uint64_t o_free[2];      // correction -> MMA and softmax i: epilogue has read O_i and m, l
-    uint64_t sm2corr[2];     // softmax i -> correction: alpha(j), j >= 1
-    uint64_t stats_full[2];  // softmax i -> correction: final m, l of the unit
+    uint64_t pv_ready[2];    // softmax i (P_i(j) written) [+ correction (O_i rescaled), d = 128] -> MMA
+    uint64_t o_done[2];      // MMA -> softmax i (d <= 64) or correction (d = 128): PV_i(j) complete
+    uint64_t o_final[2];     // MMA -> epilogue (d <= 64): the unit's last PV_i complete
+    uint64_t sm2corr[2];     // softmax i -> correction (d = 128): alpha(j), j >= 1
+    uint64_t o_free[2];      // epilogue -> MMA and softmax i: epilogue has read O_i and m, l
+    uint64_t stats_full[2];  // softmax i -> epilogue: final m, l of the unit
     uint64_t drain;
     uint64_t never;          // no arrivals: target of the injected stall
     uint64_t bias_full[2][2], bias_empty[2][2];   // [tile][stage], staged bias tiles
     uint32_t tmem_base;
     int abort_flag;
-    float alpha[2][2][kBlockM];    // [iteration parity][tile][row]
+    float alpha[2][2][kBlockM];    // [iteration parity][tile][row] (d = 128)
     float stat_m[2][2][kBlockM];   // [unit parity][tile][row]
     float stat_l[2][2][kBlockM];
 };
@@ -382,10 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh.q_empty[i], 1);
             mbar_init(&sh.s_full[i], 1);
             mbar_init(&sh.s_free[i], kBlockM);
-            mbar_init(&sh.pv_ready[i], 2 * kBlockM);
+            mbar_init(&sh.pv_ready[i], C::kPvArrivals);
             mbar_init(&sh.o_done[i], 1);
-            mbar_init(&sh.o_free[i], kBlockM);
+            mbar_init(&sh.o_final[i], 1);
             mbar_init(&sh.sm2corr[i], kBlockM);
+            mbar_init(&sh.o_free[i], kBlockM);
             mbar_init(&sh.stats_full[i], kBlockM);
         }
         for (int s = 0; s < ST; ++s) {
@@ -637,6 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                             issue_pv(0, vst, j > 0);
                             commit(&sh.o_done[0]);
+                            if (j + 1 == U.nkv0) commit(&sh.o_final[0]);
                             if (j + 1 == U.nkv0 && nkv_next[0] > 0) {
                                 if (!issue_first_s(0, nkv_next[0], kc + U.nkv1, (uit + 1) & 1))
                                     break;
@@ -651,6 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         issue_pv(1, vst, j > 0);
                         commit(&sh.o_done[1]);
                         commit(&sh.v_empty[vst]);
+                        if (j + 1 == U.nkv1) commit(&sh.o_final[1]);
                         if (j + 1 == U.nkv1 && nkv_next[1] > 0) {
                             if (!issue_first_s(1, nkv_next[1], kc + U.nkv1, (uit + 1) & 1))
                                 break;
@@ -708,8 +721,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t col_s = i ? C::kColS1 : C::kColS0;
         const uint32_t col_p = i ? C::kColP1 : C::kColP0;
+        const uint32_t col_o = i ? C::kColO1 : C::kColO0;
         const float scale_log2 = p.scale_log2;
-        const bool fast = !HAS_BIAS && !MODS && scale_log2 > 0.f;   // max over raw scores, fused scale
+        // fast path: the row maximum over raw scores and the scale fused into the exponent's FMA
+        // (no bias; of the score modifications only the left window, which only masks)
+        const bool win = MODS && p.window_left >= 0;
+        const bool fast = !HAS_BIAS && scale_log2 > 0.f && (!MODS || (p.alibi == nullptr && p.softcap <= 0.f));
         uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
         bool ok = true;
         for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
@@ -751,12 +768,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // key tiles past the end, and (causal) tiles reaching past the first row's last key
                 const bool need_mask =
                     (kv0 + kBlockN > U.Nk) || (CAUSAL && kv0 + kBlockN - 1 > first_row + U.off);
+                // left window: only a tile that starts before the window of its last row masks
+                const bool need_win = win && kv0 < first_row + kBlockM - 1 + U.off - p.window_left;
                 float m_tile;   // tile maximum, log2 domain
                 if (fast) {
-                    if (need_mask) {
+                    if (need_mask || need_win) {
                         const int lim = CAUSAL ? min(U.Nk - kv0, row + U.off - kv0 + 1) : (U.Nk - kv0);
+                        const int lo = win ? row + U.off - p.window_left - kv0 : 0;
 #pragma unroll
-                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim && c >= lo) ? s[c] : -INFINITY;
                     }
                     m_tile = row_max(s) * scale_log2;
                 } else {
@@ -815,16 +835,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int c = 0; c < kBlockN; ++c) s[c] = fmaf(-slope, fabsf(dist0 - c), s[c]);
                         }
-                        if (p.softcap > 0.f) {         // c tanh(s / c), tanh(x) = 1 - 2 / (1 + e^2x)
-                            // (both on MUFU; an FMA-pipe power of two measured slower here)
-                            const float cap = p.softcap, k2 = 2.f * kLog2e / p.softcap;
+                        if (p.softcap > 0.f) {         // c tanh(s / c): one MUFU operation per score
+                            const float cap = p.softcap, inv = 1.f / p.softcap;
 #pragma unroll
-                            for (int c = 0; c < kBlockN; ++c)
-                                s[c] = cap * (1.f - __fdividef(2.f, 1.f + ex2_approx(s[c] * k2)));
+                            for (int c = 0; c < kBlockN; ++c) s[c] = cap * tanh_approx(s[c] * inv);
                         }
                         if (p.window_left >= 0) lo = row + U.off - p.window_left - kv0;
                     }
-                    if (need_mask || (MODS && p.window_left >= 0)) {
+                    if (need_mask || need_win) {
                         const int lim = CAUSAL ? min(U.Nk - kv0, row + U.off - kv0 + 1) : (U.Nk - kv0);
 #pragma unroll
                         for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim && c >= lo) ? s[c] : -INFINITY;
@@ -840,8 +858,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_new = m_tile;
                     alpha = ex2_approx(m_ref - m_new);
                 }
-                if (!C::kSeparateP && j > 0) {
-                    // S_i(j) was issued after PV_i(j-1), so the correction has consumed alpha(j-1)
+                if (!C::kInlineRescale && j > 0) {
+                    // d = 128: S_i(j) was issued after PV_i(j-1), so the correction has consumed
+                    // alpha(j-1); it rescales O_i while the exponentials below run
                     sh.alpha[j & 1][i][t] = alpha;
                     mbar_arrive(&sh.sm2corr[i]);
                 }
@@ -852,10 +871,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float xa = fast ? scale_log2 : kLog2e;
                 const float xb = -m_use;
                 float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                // With separate P columns (d <= 64) all of P is formed first, packed in registers
+                // (s dies as P is formed), so that the wait for the previous PV_i below comes after
+                // the exponentials, not between them.  At d = 128 P goes into S_i's own columns,
+                // which nothing else reads now: each half is stored as soon as it is formed.
+                constexpr int kWords = FP8 ? 32 : 64;      // 32-bit words of this row's packed P
+                uint32_t pk[kWords];
+                auto store_p_half = [&](int half) {
+                    if constexpr (FP8)
+                        tmem_st16(tmem + lane_off + col_p + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[half * 16]));
+                    else
+                        tmem_st32(tmem + lane_off + col_p + half * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[half * 32]));
+                };
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[32];
-                    float ep0 = 0.f, ep1 = 0.f;     // e4m3: the even pair of the current 32-bit column
+                    float ep0 = 0.f, ep1 = 0.f;            // e4m3: the even pair of the current word
 #pragma unroll
                     for (int q2 = 0; q2 < 32; ++q2) {
                         const int pp = half * 32 + q2;
@@ -871,38 +901,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int q = (pp & 3) * 2;
                         fadd2_ftz(acc[q], acc[q + 1], acc[q], acc[q + 1], e0, e1);
                         if constexpr (FP8) {
-                            // four keys per 32-bit column: the even pair waits for the odd one
-                            if (q2 & 1) pk[q2 >> 1] = pack4_e4m3(ep0, ep1, e0, e1);
+                            // four keys per 32-bit word: the even pair waits for the odd one
+                            if (pp & 1) pk[pp >> 1] = pack4_e4m3(ep0, ep1, e0, e1);
                             else { ep0 = e0; ep1 = e1; }
                         } else {
-                            pk[q2] = pack2<T>(e0, e1);
+                            pk[pp] = pack2<T>(e0, e1);
                         }
                     }
-                    if constexpr (C::kSeparateP) {
-                        // P_i(j) overwrites P_i(j-1): PV_i(j-1) must have completed.  Its
-                        // completion also means the correction consumed alpha(j-1), so alpha(j)
-                        // is published only now (its barrier never runs two phases ahead).
-                        // (iteration 0 needs no wait: S_i(0) was issued after the previous unit's
-                        // last PV_i, and its commit covers that PV)
-                        if (half == 0 && j > 0) {
-                            ok = wait_phase(&sh.o_done[i], od_cnt & 1, abort_flag, p.wait_limit, p.status);
-                            ++od_cnt;
-                            ok = __all_sync(0xffffffffu, ok);
-                            if (ok) tc_fence_after();
-                        }
-                        if (half == 0 && j > 0 && ok) {
-                            sh.alpha[j & 1][i][t] = alpha;
-                            mbar_arrive(&sh.sm2corr[i]);
-                        }
-                    }
-                    if constexpr (FP8) {
-                        if (ok) tmem_st16(tmem + lane_off + col_p + half * 16, *reinterpret_cast<uint32_t(*)[16]>(pk));
-                    } else {
-                        if (ok) tmem_st32(tmem + lane_off + col_p + half * 32, pk);
+                    if constexpr (!C::kSeparateP) store_p_half(half);
+                }
+                if constexpr (C::kSeparateP) {
+                    // P_i(j) overwrites P_i(j-1), and O_i may be rescaled below: PV_i(j-1) must
+                    // have completed.  (Iteration 0 needs no wait: S_i(0) was issued after the
+                    // previous unit's last PV_i, and its commit covers that PV.)  At d = 128
+                    // S_i(j) was issued after PV_i(j-1) by the same thread, so the completion of
+                    // S_i(j), awaited above, already covers that PV.
+                    if (j > 0) {
+                        ok = wait_phase(&sh.o_done[i], od_cnt & 1, abort_flag, p.wait_limit, p.status);
+                        ++od_cnt;
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        tc_fence_after();
                     }
                 }
+                // O_i *= alpha when the reference maximum moved (rare with the threshold): each
+                // warp rescales its own 32 rows in tensor memory before releasing PV_i(j)
+                if (C::kInlineRescale && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    uint32_t r[16];               // (16-column chunks: few registers live here)
+#pragma unroll 1
+                    for (int c = 0; c < D / 16; ++c) {
+                        tmem_ld16(tmem + lane_off + col_o + c * 16, r);
+                        tmem_wait_ld16(r);
+#pragma unroll
+                        for (int q = 0; q < 16; q += 2) {
+                            float y0, y1;
+                            fmul2(y0, y1, __uint_as_float(r[q]), __uint_as_float(r[q + 1]), alpha, alpha);
+                            r[q] = __float_as_uint(y0);
+                            r[q + 1] = __float_as_uint(y1);
+                        }
+                        tmem_st16(tmem + lane_off + col_o + c * 16, r);
+                    }
+                }
+                if constexpr (C::kSeparateP) {
+                    store_p_half(0);
+                    store_p_half(1);
+                }
                 tmem_wait_st();
-                if (!ok) break;
                 const float rsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
                 l = fmaf(l, alpha, rsum);
                 m_ref = m_new;
@@ -910,9 +954,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&sh.pv_ready[i]);
             }
             if (!ok) break;
-            // The correction must have consumed the previous unit's statistics before this
-            // unit's are published: a unit with a single key tile can otherwise finish before
-            // the correction reaches the previous epilogue, running stats_full two phases ahead.
+            // The epilogue must have consumed the previous unit's statistics before this unit's
+            // are published: a unit with a single key tile can otherwise finish before the
+            // epilogue reaches the previous unit, running stats_full two phases ahead.
             if constexpr (C::kSeparateP) ++od_cnt;   // the unit's last PV_i is not waited for here
             if (uit > 0) {
                 ok = wait_phase(&sh.o_free[i], (uit - 1) & 1, abort_flag, p.wait_limit, p.status);
@@ -924,12 +968,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sh.stats_full[i]);
         }
     } else {
-        // ================================================================ correction + epilogue
-        regs_dec<C::kRegsCorrection>();
+        // ================================================================ (correction +) epilogue
+        regs_dec<C::kRegsEpilogue>();
         const int t = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         constexpr uint32_t kColO[2] = {C::kColO0, C::kColO1};
-        uint32_t c_cnt[2] = {0, 0}, st_cnt[2] = {0, 0}, od_cnt[2] = {0, 0}, uit = 0;
+        uint32_t st_cnt[2] = {0, 0}, of_cnt[2] = {0, 0}, c_cnt[2] = {0, 0}, uit = 0;
         bool ok = true;
         auto WS = [&](uint64_t* bar, uint32_t& cnt) {
             if (ok) ok = wait_phase(bar, cnt & 1, abort_flag, p.wait_limit, p.status);
@@ -937,46 +981,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             return ok;
         };
+        const bool has_next_unit_pv_arrival = !C::kInlineRescale;
         for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
             const Unit U = decode_unit<CAUSAL, MODS>(u, p);
-            for (int j = 0; ok && j < U.nkv1; ++j) {
-                for (int i = 0; i < 2; ++i) {
-                    if (j >= (i ? U.nkv1 : U.nkv0)) continue;
-                    if (j > 0) {
-                        if (!WS(&sh.sm2corr[i], c_cnt[i])) break;
-                        const float alpha = sh.alpha[j & 1][i][t];
-                        if (!WS(&sh.o_done[i], od_cnt[i])) break;   // PV_i(j-1) complete
-                        tc_fence_after();
-                        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                            uint32_t r[32];
+            if constexpr (!C::kInlineRescale) {
+                // d = 128, the correction: O_i *= alpha(j) between PV_i(j-1) and PV_i(j) (only when
+                // some row of the warp moved its reference maximum), then its pv_ready arrival.
+                // Its o_done waits use the of_cnt counters: every PV_i phase, the last one in the
+                // epilogue below.
+                for (int j = 0; ok && j < U.nkv1; ++j) {
+                    for (int i = 0; i < 2; ++i) {
+                        if (j >= (i ? U.nkv1 : U.nkv0)) continue;
+                        if (j > 0) {
+                            if (!WS(&sh.sm2corr[i], c_cnt[i])) break;
+                            const float alpha = sh.alpha[j & 1][i][t];
+                            if (!WS(&sh.o_done[i], of_cnt[i])) break;   // PV_i(j-1) complete
+                            tc_fence_after();
+                            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                                uint32_t r[32];
 #pragma unroll
-                            for (int c = 0; c < D / 32; ++c) {
-                                tmem_ld32(tmem + lane_off + kColO[i] + c * 32, r);
-                                tmem_wait_ld(r);
+                                for (int c = 0; c < D / 32; ++c) {
+                                    tmem_ld32(tmem + lane_off + kColO[i] + c * 32, r);
+                                    tmem_wait_ld(r);
 #pragma unroll
-                                for (int q = 0; q < 32; q += 2) {
-                                    float x0, x1;
-                                    fmul2(x0, x1, __uint_as_float(r[q]), __uint_as_float(r[q + 1]), alpha, alpha);
-                                    r[q] = __float_as_uint(x0);
-                                    r[q + 1] = __float_as_uint(x1);
+                                    for (int q = 0; q < 32; q += 2) {
+                                        float x0, x1;
+                                        fmul2(x0, x1, __uint_as_float(r[q]), __uint_as_float(r[q + 1]), alpha, alpha);
+                                        r[q] = __float_as_uint(x0);
+                                        r[q + 1] = __float_as_uint(x1);
+                                    }
+                                    tmem_st32(tmem + lane_off + kColO[i] + c * 32, r);
                                 }
-                                tmem_st32(tmem + lane_off + kColO[i] + c * 32, r);
+                                tmem_wait_st();
                             }
-                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(&sh.pv_ready[i]);
+                        } else if (uit == 0) {
+                            mbar_arrive(&sh.pv_ready[i]);   // later units: arrived by the previous epilogue
                         }
-                        tc_fence_before();
-                        mbar_arrive(&sh.pv_ready[i]);
-                    } else if (uit == 0) {
-                        mbar_arrive(&sh.pv_ready[i]);   // later units: arrived by the previous epilogue
                     }
                 }
+                if (!ok) break;
             }
-            if (!ok) break;
-            // epilogue: O = O_acc / l (* sigmoid(G)), lse = (m + log2 l) * ln 2.
-            // O_i is released as soon as its last chunk is in registers, together with the next
-            // unit's first pv_ready arrival (iteration 0 needs no rescale), so the next unit's
-            // PV_i(0) does not wait for the gate arithmetic and global stores.
-            const bool has_next = unit_at(uit + 1) < p.num_units;
+            // O = O_acc / l (* sigmoid(G)), lse = (m + log2 l) * ln 2.  O_i is released as soon as
+            // its last chunk is in registers (at d = 128 together with the next unit's first
+            // pv_ready arrival: iteration 0 needs no rescale), so the next unit's PV_i(0) does not
+            // wait for the gate arithmetic and the global stores.
+            const bool has_next = has_next_unit_pv_arrival && unit_at(uit + 1) < p.num_units;
             for (int i = 0; i < 2; ++i) {
                 const int row = U.q0 + i * kBlockM + t;
                 const bool row_ok = row < U.N;
@@ -995,7 +1046,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (!WS(&sh.stats_full[i], st_cnt[i])) break;  // final m, l
-                if (!WS(&sh.o_done[i], od_cnt[i])) break;      // last PV_i complete
+                // the unit's last PV_i complete (d = 128: the last phase of o_done)
+                if (!WS(C::kInlineRescale ? &sh.o_final[i] : &sh.o_done[i], of_cnt[i])) break;
                 tc_fence_after();
                 const float m = sh.stat_m[uit & 1][i][t];
                 const float l = sh.stat_l[uit & 1][i][t];
@@ -1015,7 +1067,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             else raw = __ldg(reinterpret_cast<const uint4*>(grow + c * 32 + v8 * 8));
                             const T* e = reinterpret_cast<const T*>(&raw);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) o[q] *= 1.f / (1.f + ex2_approx(-to_f32<T>(e[q]) * kLog2e));
+                            // sigmoid(g) = (1 + tanh(g / 2)) / 2: one MUFU operation per element
+                            for (int q = 0; q < 8; ++q) o[q] *= fmaf(0.5f, tanh_approx(0.5f * to_f32<T>(e[q])), 0.5f);
                         }
                         uint4 w;
                         w.x = pack2<T>(o[0], o[1]);

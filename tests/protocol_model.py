@@ -1,7 +1,7 @@
 """A model of the forward kernel's mbarrier protocol, checked under random interleavings.
 
 The kernel in exact_attention_sdpa_b200/csrc/attn_fwd_kernel.cuh moves every tile between its
-roles (TMA producer, MMA issuer, two softmax warpgroups, correction warpgroup) through
+roles (TMA producer, MMA issuer, two softmax warpgroups, epilogue warpgroup) through
 mbarriers whose waits name a phase only by its parity.  compute-sanitizer cannot run on the
 machines these kernels are measured on, so this module re-states the protocol as it is written
 in the kernel, one actor per warp, and executes it on the CPU under random schedules:
@@ -14,7 +14,7 @@ in the kernel, one actor per warp, and executes it on the CPU under random sched
     different threads execute in any order;
   * TMA loads complete in any order and then arrive on their barrier;
   * every buffer (Q, K, V and bias stages in shared memory; S, P, O columns in tensor memory;
-    the alpha and statistics slots) carries a version tag, and every read checks that it sees
+    the statistics slots) carries a version tag, and every read checks that it sees
     exactly the version the kernel means to read.
 
 A run fails on a stale or early read (a race), on a wait that returns while its barrier is not
@@ -129,10 +129,13 @@ class State:
         self.v_empty = [B(f"v_empty{s}", 1) for s in range(ST)]
         self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
         self.s_free = [B(f"s_free{i}", 128) for i in range(2)]
-        self.pv_ready = [B(f"pv_ready{i}", 256) for i in range(2)]
+        # separate P (d <= 64): the softmax rescales O itself and alone releases PV_i(j); P inside S
+        # (d = 128): the correction warpgroup rescales O and releases PV_i(j) with the softmax
+        self.pv_ready = [B(f"pv_ready{i}", 128 if cfg.separate_p else 256) for i in range(2)]
         self.o_done = [B(f"o_done{i}", 1) for i in range(2)]
-        self.o_free = [B(f"o_free{i}", 128) for i in range(2)]
+        self.o_final = [B(f"o_final{i}", 1) for i in range(2)]
         self.sm2corr = [B(f"sm2corr{i}", 128) for i in range(2)]
+        self.o_free = [B(f"o_free{i}", 128) for i in range(2)]
         self.stats_full = [B(f"stats_full{i}", 128) for i in range(2)]
         self.bias_full = [[B(f"bias_full{i}.{s}", 1) for s in range(BS)] for i in range(2)]
         self.bias_empty = [[B(f"bias_empty{i}.{s}", 128) for s in range(BS)] for i in range(2)]
@@ -148,8 +151,8 @@ class State:
         self.tS = [[None] * 4 for _ in range(2)]      # S_i (and P_i at d = 128)
         self.tP = [[None] * 4 for _ in range(2)]      # P_i (d <= 64)
         self.tO = [[None] * 4 for _ in range(2)]      # O_i: dict(unit, done, rescaled, read)
-        self.alpha = [[[None] * 4 for _ in range(2)] for _ in range(2)]   # [j parity][tile][quarter]
         self.stats = [[[None] * 4 for _ in range(2)] for _ in range(2)]   # [unit parity][tile][quarter]
+        self.alpha = [[[None] * 4 for _ in range(2)] for _ in range(2)]   # [j parity][tile][quarter] (d = 128)
 
     def expect(self, what: str, got, want) -> None:
         if got != want:
@@ -363,6 +366,8 @@ def mma_issuer(st: State):
                         break
                     yield pv_mma(st, 0, k, j, vst, vn)
                     yield Commit("mma", st.o_done[0])
+                    if j + 1 == n0:
+                        yield Commit("mma", st.o_final[0])
                     if j + 1 == n0 and nxt[0] > 0:
                         if not (yield from first_s(0, k + 1, kc + n1, nxt[0])):
                             break
@@ -377,6 +382,8 @@ def mma_issuer(st: State):
                 yield pv_mma(st, 1, k, j, vst, vn)
                 yield Commit("mma", st.o_done[1])
                 yield Commit("mma", st.v_empty[vst])
+                if j + 1 == n1:
+                    yield Commit("mma", st.o_final[1])
                 if j + 1 == n1 and nxt[1] > 0:
                     if not (yield from first_s(1, k + 1, kc + n1, nxt[1])):
                         break
@@ -464,31 +471,43 @@ def softmax_warp(st: State, i: int, q: int):
                 yield Arrive(st.bias_empty[i][bst], 32)
                 bcnt += 1
 
-            def put_alpha(s, k=k, j=j):
-                s.alpha[j & 1][i][q] = (k, j)
             if not cfg.separate_p and j > 0:
+                # d = 128: alpha(j) for the correction (S_i(j) was issued after PV_i(j-1), so the
+                # correction has consumed alpha(j-1))
+                def put_alpha(s, k=k, j=j):
+                    s.alpha[j & 1][i][q] = (k, j)
                 yield Do("alpha", put_alpha)
                 yield Arrive(st.sm2corr[i], 32)
-            if cfg.separate_p and j > 0:
-                if cfg.plant == "alpha_before_o_done":
-                    yield Do("alpha", put_alpha)
-                    yield Arrive(st.sm2corr[i], 32)
+            if cfg.separate_p and j > 0 and cfg.plant != "rescale_before_o_done":
+                # P_i(j) overwrites P_i(j-1) and O_i may be rescaled: PV_i(j-1) must be complete
                 if cfg.plant != "no_o_done_wait":
                     ok = yield Wait(st.o_done[i], od_cnt & 1, od_cnt)
                 od_cnt += 1
-                if ok and cfg.plant != "alpha_before_o_done":
-                    yield Do("alpha", put_alpha)
-                    yield Arrive(st.sm2corr[i], 32)
+
+            def rescale(s, k=k, j=j):
+                o = s.tO[i][q]
+                s.expect(f"softmax{i}.{q} rescales O{i}", None if o is None else (o["unit"], o["done"]), (k, j - 1))
+                o["rescaled"] = j
 
             def write_p(s, k=k, j=j):
                 if s.cfg.separate_p:
                     s.tP[i][q] = ("P", k, j)
                 else:
                     s.tS[i][q] = ("P", k, j)
-            if ok:
-                yield Do("st P", write_p)
             if not ok:
                 break
+            if cfg.plant == "pv_ready_before_rescale" and j > 0 and cfg.separate_p:
+                yield Arrive(st.pv_ready[i], 32)
+            if j > 0 and cfg.separate_p:
+                yield Do("rescale O", rescale)
+            if cfg.separate_p and j > 0 and cfg.plant == "rescale_before_o_done":
+                ok = yield Wait(st.o_done[i], od_cnt & 1, od_cnt)
+                od_cnt += 1
+                if not ok:
+                    break
+            yield Do("st P", write_p)
+            if cfg.plant == "pv_ready_before_rescale" and j > 0 and cfg.separate_p:
+                continue
             yield Arrive(st.pv_ready[i], 32)
         if not ok:
             break
@@ -506,10 +525,13 @@ def softmax_warp(st: State, i: int, q: int):
     yield from teardown(st)
 
 
-def correction_warp(st: State, q: int):
-    """Warp q of the correction warpgroup: rescale O_i for alpha(j), then the epilogue."""
+def epilogue_warp(st: State, q: int):
+    """Warp q of warpgroup 2.  With separate P (d <= 64) the epilogue alone: per unit and tile the
+    final statistics and the last PV_i (o_final), then O_i is read and released.  At d = 128 also
+    the correction: O_i rescaled for alpha(j) between PV_i(j-1) and PV_i(j), its pv_ready
+    arrivals, and the epilogue on o_done's last phase."""
     cfg = st.cfg
-    c_cnt, st_cnt, od_cnt = [0, 0], [0, 0], [0, 0]
+    st_cnt, of_cnt, c_cnt = [0, 0], [0, 0], [0, 0]
     n_units = len(cfg.units)
     ok = True
 
@@ -523,40 +545,41 @@ def correction_warp(st: State, q: int):
     for k, (n0, n1) in enumerate(cfg.units):
         if not ok:
             break
-        j = 0
-        while ok and j < n1:
-            for i in range(2):
-                if j >= (n1 if i else n0):
-                    continue
-                if j > 0:
-                    if not (yield from WS(st.sm2corr[i], c_cnt, i)):
-                        break
+        if not cfg.separate_p:
+            j = 0
+            while ok and j < n1:
+                for i in range(2):
+                    if j >= (n1 if i else n0):
+                        continue
+                    if j > 0:
+                        if not (yield from WS(st.sm2corr[i], c_cnt, i)):
+                            break
 
-                    def read_alpha(s, k=k, j=j, i=i):
-                        s.expect(f"correction.{q} reads alpha{i}", s.alpha[j & 1][i][q], (k, j))
-                    yield Do("alpha", read_alpha)
-                    if not (yield from WS(st.o_done[i], od_cnt, i)):
-                        break
+                        def read_alpha(s, k=k, j=j, i=i):
+                            s.expect(f"correction.{q} reads alpha{i}", s.alpha[j & 1][i][q], (k, j))
+                        yield Do("alpha", read_alpha)
+                        if not (yield from WS(st.o_done[i], of_cnt, i)):
+                            break
 
-                    def rescale(s, k=k, j=j, i=i):
-                        o = s.tO[i][q]
-                        s.expect(f"correction.{q} rescales O{i}", (o["unit"], o["done"]), (k, j - 1))
-                        o["rescaled"] = j
-                    if cfg.plant == "arrive_before_rescale":
+                        def rescale(s, k=k, j=j, i=i):
+                            o = s.tO[i][q]
+                            s.expect(f"correction.{q} rescales O{i}", (o["unit"], o["done"]), (k, j - 1))
+                            o["rescaled"] = j
+                        if cfg.plant == "arrive_before_rescale":
+                            yield Arrive(st.pv_ready[i], 32)
+                        yield Do("rescale O", rescale)
+                        if cfg.plant != "arrive_before_rescale":
+                            yield Arrive(st.pv_ready[i], 32)
+                    elif k == 0:
                         yield Arrive(st.pv_ready[i], 32)
-                    yield Do("rescale O", rescale)
-                    if cfg.plant != "arrive_before_rescale":
-                        yield Arrive(st.pv_ready[i], 32)
-                elif k == 0:
-                    yield Arrive(st.pv_ready[i], 32)
-            j += 1
-        if not ok:
-            break
-        has_next = k + 1 < n_units
+                j += 1
+            if not ok:
+                break
+        has_next = k + 1 < n_units and not cfg.separate_p
         for i in range(2):
             if not (yield from WS(st.stats_full[i], st_cnt, i)):
                 break
-            if not (yield from WS(st.o_done[i], od_cnt, i)):
+            if not (yield from WS(st.o_final[i] if cfg.separate_p else st.o_done[i], of_cnt, i)):
                 break
             last = (n1 if i else n0) - 1
 
@@ -578,7 +601,7 @@ def kernel_roles(st: State) -> dict:
         for q in range(4):
             roles[f"softmax{i}.{q}"] = softmax_warp(st, i, q)
     for q in range(4):
-        roles[f"corr.{q}"] = correction_warp(st, q)
+        roles[f"epi.{q}"] = epilogue_warp(st, q)
     return roles
 
 

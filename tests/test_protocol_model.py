@@ -54,7 +54,7 @@ def test_single_tile_units_back_to_back():
         pm.run(cfg, seed=rep)
 
 
-ROLES = ["tma", "mma"] + [f"softmax{i}.{q}" for i in range(2) for q in range(4)] + [f"corr.{q}" for q in range(4)]
+ROLES = ["tma", "mma"] + [f"softmax{i}.{q}" for i in range(2) for q in range(4)] + [f"epi.{q}" for q in range(4)]
 
 
 @pytest.mark.parametrize("sep,causal,stages,bias", [(True, True, 3, 0), (True, False, 4, 2), (True, True, 3, 1),
@@ -94,10 +94,10 @@ PLANTS = {
     "empty_parity": True,           # producer waits the K/V release of the wrong phase
     "no_s_free_wait": True,         # S_0(j+1) issued before the softmax read S_0(j)
     "s_before_pv": False,           # d = 128: S_0(j+1) overwrites P_0(j) before PV_0(j)
-    "alpha_before_o_done": True,    # alpha(j) published before PV_i(j-1) completed
+    "rescale_before_o_done": True,  # O_i rescaled before PV_i(j-1) completed
     "no_o_done_wait": True,         # P_i(j) written while PV_i(j-1) may still read P_i(j-1)
-    "stats_no_o_free_wait": True,   # final m, l published before the previous epilogue read them
-    "arrive_before_rescale": True,  # correction releases PV_i(j) before rescaling O_i
+    "pv_ready_before_rescale": True,   # softmax releases PV_i(j) before rescaling O_i (d <= 64)
+    "arrive_before_rescale": False,    # correction releases PV_i(j) before rescaling O_i (d = 128)
 }
 
 
@@ -116,6 +116,20 @@ def test_model_finds_planted_mistakes(plant):
     pytest.fail(f"planted mistake {plant!r} went unnoticed in 400 schedules")
 
 
+def test_softmax_o_free_wait_is_a_second_guard():
+    """The softmax's wait for the previous epilogue (o_free) before it publishes a unit's final
+    m, l is implied by the rest of the protocol: the next unit's first S_i is issued only after
+    PV_i(0) of the current unit, which waited for the epilogue two units back.  Without the wait
+    the model still finds no stale read; the kernel keeps it as a cheap second guard."""
+    for rep in range(200):
+        rng = random.Random(rep)
+        sep = rep % 2 == 0
+        cfg = pm.Config(separate_p=sep, causal=True, stages=3 if sep else 2,
+                        units=pm.random_units(rng, True, rng.randint(2, 6), max_tiles=2),
+                        plant="stats_no_o_free_wait")
+        pm.run(cfg, seed=rep)
+
+
 def test_model_barriers_match_the_kernel_source():
     # The model must know every mbarrier the kernel initialises, with the same arrival count;
     # a barrier added to or re-counted in the kernel without the model fails here.
@@ -123,11 +137,16 @@ def test_model_barriers_match_the_kernel_source():
     import re
     src = open(os.path.join(os.path.dirname(__file__), "..", "exact_attention_sdpa_b200", "csrc",
                             "attn_fwd_kernel.cuh")).read()
-    found = {}
-    for name, expr in re.findall(r"mbar_init\(&sh\.(\w+)(?:\[[^\]]*\])*,\s*([^;]+)\);", src):
-        found[name] = eval(expr.strip(), {"kBlockM": 128})
-    found.pop("never")            # stall-injection target: nothing ever arrives on it
-    st = pm.State(pm.Config(units=[(1, 1)], bias_stages=1))
+    for sep in (True, False):
+        found = {}
+        for name, expr in re.findall(r"mbar_init\(&sh\.(\w+)(?:\[[^\]]*\])*,\s*([^;]+)\);", src):
+            # C::kPvArrivals: the softmax's 128 arrivals, plus the correction's 128 at d = 128
+            found[name] = eval(expr.strip().replace("C::kPvArrivals", "kPv"), {"kBlockM": 128, "kPv": 128 if sep else 256})
+        found.pop("never")            # stall-injection target: nothing ever arrives on it
+        check_barriers(found, pm.State(pm.Config(units=[(1, 1)], bias_stages=1, separate_p=sep)))
+
+
+def check_barriers(found, st):
     model = {}
     for name, val in vars(st).items():
         bars = val
