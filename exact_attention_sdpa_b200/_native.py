@@ -18,12 +18,14 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libattn.so")
 
-ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_CHECK = range(6)
+ATTN_BUILD_DEBUG_CHECKS = 1
+DEBUG_LIB_PATH = os.path.join(_PKG, "libattn_debug.so")
 ATTN_F16, ATTN_BF16, ATTN_F32, ATTN_E4M3 = 0, 1, 2, 3
 
 # every function include/attn.h declares
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_fwd_fp8", "attn_bwd", "attn_bwd_ex", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
-            "attn_debug_inject_stall", "attn_debug_exp2", "attn_version")
+            "attn_debug_inject_stall", "attn_debug_exp2", "attn_build_flags", "attn_version")
 
 
 class AttnTensor(ctypes.Structure):
@@ -88,6 +90,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_debug_exp2.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
                                         ctypes.c_void_p]
         lib.attn_debug_exp2.restype = ctypes.c_int
+        lib.attn_build_flags.argtypes = []
+        lib.attn_build_flags.restype = ctypes.c_int
         lib.attn_version.argtypes = []
         lib.attn_version.restype = ctypes.c_char_p
         if path is None:

@@ -1,6 +1,9 @@
 """Builds libattn.so in-tree with nvcc for sm_100a (no JIT cache, no torch extension).
 
-    python -m exact_attention_sdpa_b200.build [--force] [--verbose]
+    python -m exact_attention_sdpa_b200.build [--force] [--verbose] [--debug]
+
+--debug builds libattn_debug.so: the same kernels with their device-side index and range
+checks compiled in (status ATTN_ERR_CHECK instead of a fault).
 """
 from __future__ import annotations
 
@@ -13,6 +16,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libattn.so")
+DEBUG_LIB = os.path.join(PKG, "libattn_debug.so")
 SOURCES = [os.path.join(PKG, "csrc", "attn_api.cu")]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -32,21 +36,24 @@ def _inputs():
     return sorted(files)
 
 
-def is_stale() -> bool:
-    """True when libattn.so is missing or older than any CUDA source or public header."""
-    if not os.path.exists(LIB):
+def is_stale(lib: str = LIB) -> bool:
+    """True when the library is missing or older than any CUDA source or public header."""
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libattn.so in the package directory for sm_100a (when stale or forced); returns its
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile libattn.so (or, with debug=True, libattn_debug.so: the device-side index and range
+    checks compiled in) in the package directory for sm_100a, when stale or forced; returns its
     path.  Raises RuntimeError with nvcc's output if the compilation fails."""
-    if not force and not is_stale():
-        return LIB
+    out = DEBUG_LIB if debug else LIB
+    if not force and not is_stale(out):
+        return out
     cmd = [nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-           "-I" + os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *SOURCES]
+           "-I" + os.path.join(ROOT, "include"), *(["-DATTN_DEBUG=1"] if debug else []), "-o", out + ".tmp",
+           *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -55,10 +62,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         print(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    path = build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
+    path = build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv)
     print(path)

@@ -843,6 +843,7 @@ const char* attn_status_string(attn_status_t status) {
         case ATTN_ERR_UNSUPPORTED: return "unsupported (fp32, mixed dtypes, or head dim not in {32, 64, 128})";
         case ATTN_ERR_CUDA: return "CUDA error (launch, tensor-map encoding or device query failed)";
         case ATTN_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        case ATTN_ERR_CHECK: return "a debug build's device-side index or range check failed";
         default: return "unknown status";
     }
 }
@@ -855,14 +856,17 @@ attn_status_t attn_last_device_status(cudaStream_t stream) {
     if (cudaMemcpyFromSymbolAsync(&v, g_status_read, sizeof(v), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
         return ATTN_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
-    return (v & attn::kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+    if (v & attn::kStatusTimeout) return ATTN_ERR_TIMEOUT;
+    return (v & attn::kStatusCheck) ? ATTN_ERR_CHECK : ATTN_OK;
 }
 
 void attn_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles < 1024 ? 1024 : cycles; }
 
 void attn_debug_inject_stall(int enable) { g_inject_stall = enable != 0; }
 
-const char* attn_version(void) { return "0.1.0"; }
+const char* attn_version(void) { return "0.2.0"; }
+
+int attn_build_flags(void) { return ATTN_DEBUG ? ATTN_BUILD_DEBUG_CHECKS : 0; }
 
 }  // extern "C"
 

@@ -34,6 +34,7 @@ namespace bwdtc {
 constexpr int kThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusCheck = 2u;     // debug builds: an index or range check failed (ATTN_CHECK)
 constexpr unsigned long long kDrainLimit = 1ull << 32;
 
 struct Params {
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         m_end = last_q < 0 ? 0 : min(nqb, last_q / 64 + 1);
     }
     const int nit = m_end > m0 ? m_end - m0 : 0;
+    ATTN_CHECK(p.status, m0 >= 0 && m0 <= nqb && m_end >= 0 && m_end <= nqb && k0 < p.Nk && b < p.B);
 
     if (t == 0) {
         mbar_init(&bar_kv, 1);
@@ -275,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    ATTN_CHECK(p.status, (tmem >> 16) == 0u && (tmem & 0xFFFFu) + C::kCols <= 512u);
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     int* abort_p = &abort_flag;
 
@@ -488,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int lo_key = q0 + p.causal_off - p.window_left;
         kb_first = lo_key > 0 ? min(nkb, lo_key / 64) : 0;
     }
+    ATTN_CHECK(p.status, kb_first >= 0 && kb_first <= nkb && nkb <= nkb_all && q0 < p.N + 127 && b < p.B);
 
     if (t == 0) {
         mbar_init(&bar_q, 1);
@@ -508,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    ATTN_CHECK(p.status, (tmem >> 16) == 0u && (tmem & 0xFFFFu) + C::kCols <= 512u);
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     int* abort_p = &abort_flag;
 

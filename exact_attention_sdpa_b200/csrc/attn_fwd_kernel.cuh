@@ -63,6 +63,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f; // log2 domain: rescale only when m grows by > 2^8
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusCheck = 2u;     // debug builds: an index or range check failed
+
 constexpr unsigned long long kDrainLimit = 1ull << 32;
 constexpr int kMaxSeq = 64;    // sequences of a ragged batch handled by one launch
 
@@ -356,6 +358,11 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
         U.nkv0 -= U.kv_lo;
         U.nkv1 -= U.kv_lo;
     }
+    ATTN_CHECK(p.status, U.b >= 0 && U.b < p.B && U.h >= 0 && U.h < p.H && U.qp >= 0 && U.q0 < U.N);
+    ATTN_CHECK(p.status, U.kv_lo >= 0 && U.nkv0 >= 1 && U.nkv1 >= U.nkv0 && U.nkv1 <= U.nkv0 + 1);
+    ATTN_CHECK(p.status, (U.kv_lo + U.nkv1 - 1) * kBlockN < U.Nk || U.nkv1 == 1);
+    ATTN_CHECK(p.status, U.q_base >= 0 && U.k_base >= 0 && U.q_base + U.N <= (p.n_seq > 0 ? p.N : U.N) &&
+                             U.k_base + U.Nk <= (p.n_seq > 0 ? p.Nk : U.Nk));
     return U;
 }
 
@@ -425,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
     int* abort_flag = &sh.abort_flag;
+    ATTN_CHECK(p.status, tmem == 0u);      // all 512 columns, from lane 0 column 0
 
     if (wg == 3) {
         regs_dec<C::kRegsOther>();
@@ -479,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t st = cnt % ST;
                 if (cnt >= ST && !WU(&empty[st], ((cnt / ST) - 1) & 1)) return;
                 const int key0 = U.k_base + (U.kv_lo + j) * kBlockN;
+                ATTN_CHECK(p.status, key0 >= 0 && (C::kAtomCols * C::kElemBytes) % 16 == 0 && (!FP8 || key0 % 16 == 0));
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&full[st], C::kTileBytes);
                     if (FP8 && ring == sV) {
@@ -496,14 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             for (int k = 0, u = unit_at(0); ok && u < p.num_units; u = unit_at(++k)) {
                 const Unit U = decode_unit<CAUSAL, MODS>(u, p);
-                load_q(0, U);
+                // the unit's first bias tiles go first: their stages free up as soon as the
+                // softmax has read the previous unit's first tiles, long before the Q slots do
+                // (each Q_i waits for the previous unit's last S_i)
+                if constexpr (BC::kTma) {
+                    load_bias(0, 0, U);
+                    if (ok) load_bias(1, 0, U);
+                }
+                if (ok) load_q(0, U);
                 if (ok) load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, 0, U);
                 if (ok) load_q(1, U);
                 if (ok) load_kv(sh.v_full, sh.v_empty, sV, &tm_v, vc, 0, U);
-                if constexpr (BC::kTma) {
-                    if (ok) load_bias(0, 0, U);
-                    if (ok) load_bias(1, 0, U);
-                }
                 for (int j = 1; ok && j < U.nkv1; ++j) {
                     load_kv(sh.k_full, sh.k_empty, sK, &tm_k, kc, j, U);
                     if (ok) load_kv(sh.v_full, sh.v_empty, sV, &tm_v, vc, j, U);
@@ -1090,6 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     finish_chunk(r, c);
                 }
+                ATTN_CHECK(p.status, !row_ok || (U.q_base + row >= 0 && U.q_base + row < (p.n_seq > 0 ? p.N : U.N)));
                 if (p.lse != nullptr && row_ok)
                     p.lse[U.b * p.lse_sb + U.h * p.lse_sh + U.q_base + row] =
                         (l > 0.f) ? (m + lg2_approx(l)) * kLn2 : -INFINITY;

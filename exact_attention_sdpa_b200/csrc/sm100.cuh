@@ -9,6 +9,24 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+// Debug builds (compiled with -DATTN_DEBUG=1: libattn_debug.so) check the indices and ranges the
+// kernels derive (work-unit decode, tile coordinates, tensor-memory columns, output rows) and
+// record a failure as bit 2 of the device status word instead of faulting; release builds
+// compile the checks away.
+#ifndef ATTN_DEBUG
+#define ATTN_DEBUG 0
+#endif
+#if ATTN_DEBUG
+#define ATTN_CHECK(status, cond)                         \
+    do {                                                 \
+        if (!(cond)) atomicOr((status), 2u);             \
+    } while (0)
+#else
+#define ATTN_CHECK(status, cond) \
+    do {                         \
+    } while (0)
+#endif
+
 namespace attn {
 namespace sm100 {
 

@@ -39,7 +39,8 @@ typedef enum {
     ATTN_ERR_INVALID_ARG = 1,   /* null pointer, shape/stride mismatch, misalignment, non-finite scale */
     ATTN_ERR_UNSUPPORTED = 2,   /* a valid request this kernel does not implement (fp32, head dim, ...) */
     ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call or the launch failed */
-    ATTN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (status word, see below) */
+    ATTN_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (status word, see below) */
+    ATTN_ERR_CHECK = 5          /* debug builds only: a device-side index or range check failed */
 } attn_status_t;
 
 typedef enum {
@@ -238,8 +239,10 @@ const char* attn_status_string(attn_status_t status);
  * of a kernel still running on another stream may therefore be reported by
  * this call, or by a later one, instead of the caller whose launch it was;
  * callers that run the library on several streams and need per-call status
- * must serialise their reads.  Returns ATTN_OK, ATTN_ERR_TIMEOUT, or
- * ATTN_ERR_CUDA if the exchange, the read or the synchronisation failed.
+ * must serialise their reads.  Returns ATTN_OK, ATTN_ERR_TIMEOUT, ATTN_ERR_CHECK
+ * (a debug build's device-side index or range check failed; see
+ * attn_build_flags), or ATTN_ERR_CUDA if the exchange, the read or the
+ * synchronisation failed.
  */
 attn_status_t attn_last_device_status(cudaStream_t stream);
 
@@ -322,6 +325,17 @@ attn_status_t attn_fwd_fp8(const attn_tensor_t* q, const attn_tensor_t* k, const
  */
 enum { ATTN_EXP2_FMA_PIPE = 0, ATTN_EXP2_MUFU = 1, ATTN_EXP2_CUDA_EXP2F = 2 };
 attn_status_t attn_debug_exp2(const float* x, float* y, int64_t n, int mode, cudaStream_t stream);
+
+/*
+ * attn_build_flags -- how this library was built.  ATTN_BUILD_DEBUG_CHECKS: the
+ * debug build (libattn_debug.so, compiled with -DATTN_DEBUG=1).  Its kernels check
+ * the indices and ranges they derive (the work-unit decode, tile coordinates and
+ * their 16-byte alignment, the tensor-memory allocation, output rows) and record a
+ * failure in the device status word (ATTN_ERR_CHECK from attn_last_device_status)
+ * instead of faulting; results are otherwise the release build's.
+ */
+enum { ATTN_BUILD_DEBUG_CHECKS = 1 };
+int attn_build_flags(void);
 
 /* The library version as "major.minor.patch" (static string). */
 const char* attn_version(void);

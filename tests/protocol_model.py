@@ -175,7 +175,7 @@ def teardown(st: State):
 
 
 def producer(st: State):
-    """TMA producer warp: Q0, K(0), Q1, V(0), [bias], then K(j), V(j), [bias] per unit; drains."""
+    """TMA producer warp: [bias(0)], Q0, K(0), Q1, V(0), then K(j), V(j), [bias(j)] per unit; drains."""
     cfg, ST, BS = st.cfg, st.cfg.stages, st.cfg.bias_stages
     cnt = {"K": 0, "V": 0}
     qc = [0, 0]
@@ -224,18 +224,18 @@ def producer(st: State):
     for k, (n0, n1) in enumerate(cfg.units):
         if not ok:
             break
-        yield from load_q(0, k)
+        if BS:                             # the unit's first bias tiles go first
+            yield from load_bias(0, 0, k)
+            if ok:
+                yield from load_bias(1, 0, k)
+        if ok:
+            yield from load_q(0, k)
         if ok:
             yield from load_kv("K")
         if ok:
             yield from load_q(1, k)
         if ok:
             yield from load_kv("V")
-        if BS:
-            if ok:
-                yield from load_bias(0, 0, k)
-            if ok:
-                yield from load_bias(1, 0, k)
         j = 1
         while ok and j < n1:
             yield from load_kv("K")
