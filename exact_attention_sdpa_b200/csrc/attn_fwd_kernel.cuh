@@ -643,9 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (j + 1 < U.nkv1) {
                             if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
                             ++sf_cnt[1];
-                            // (without causal masking both tiles have the same key tiles, and
-                            // S0(j+1) has just waited for this one)
-                            if (CAUSAL && !W(&sh.k_full[kst], kph)) break;
+                            // (K(j+1) has been waited for by S0(j+1) unless tile 0 ends at j: only
+                            // causal units give tile 1 one more key tile)
+                            if (j + 1 >= U.nkv0 && !W(&sh.k_full[kst], kph)) break;
                             tc_fence_after();
                             issue_s(1, kst);
                             commit(&sh.s_full[1]);
@@ -670,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
                         ++pv_cnt[1];
                         if (j == 0 && uit > 0 && !W(&sh.o_free[1], (uit - 1) & 1)) break;
-                        if (CAUSAL && !W(&sh.v_full[vst], vph)) break;   // else seen by PV0(j)
+                        if (j >= U.nkv0 && !W(&sh.v_full[vst], vph)) break;   // else seen by PV0(j)
                         tc_fence_after();
                         issue_pv(1, vst, j > 0);
                         commit(&sh.o_done[1]);

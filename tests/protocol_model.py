@@ -103,6 +103,7 @@ class Config:
     units: list = field(default_factory=list)    # per unit (nkv0, nkv1)
     plant: str = ""               # a protocol mistake planted on purpose (tests of the checker)
     timeout: tuple = ()           # (role, n): that role's n-th bounded wait gives up (abort path)
+    tma_weight: float = 1.0       # relative chance that a pending TMA load completes next (< 1: slow loads)
 
 
 def random_units(rng: random.Random, causal: bool, n_units: int, max_tiles: int = 5) -> list:
@@ -349,7 +350,7 @@ def mma_issuer(st: State):
                     if not (yield from W(st.s_free[1], sf_cnt[1] & 1, sf_cnt[1])):
                         break
                     sf_cnt[1] += 1
-                    if cfg.causal and not (yield from W(st.k_full[kst], kph, kn // ST)):
+                    if j + 1 >= n0 and cfg.plant != "s1_skips_k_wait" and not (yield from W(st.k_full[kst], kph, kn // ST)):
                         break
                     yield s_mma(st, 1, k, j + 1, kst, kn)
                     yield Commit("mma", st.s_full[1])
@@ -377,7 +378,7 @@ def mma_issuer(st: State):
                 pv_cnt[1] += 1
                 if j == 0 and k > 0 and not (yield from W(st.o_free[1], (k - 1) & 1, k - 1)):
                     break
-                if cfg.causal and not (yield from W(st.v_full[vst], vph, vn // ST)):
+                if j >= n0 and not (yield from W(st.v_full[vst], vph, vn // ST)):
                     break
                 yield pv_mma(st, 1, k, j, vst, vn)
                 yield Commit("mma", st.o_done[1])
@@ -658,7 +659,11 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
             if info is not None:
                 info["aborted"] = st.abort
             return steps
-        kind, key = rng.choice(choices)
+        if cfg.tma_weight != 1.0:
+            weights = [cfg.tma_weight if c[0] == "tma" else 1.0 for c in choices]
+            kind, key = rng.choices(choices, weights)[0]
+        else:
+            kind, key = rng.choice(choices)
         steps += 1
         if steps > max_steps:
             fail("step limit")
