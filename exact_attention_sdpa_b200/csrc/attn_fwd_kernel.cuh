@@ -557,38 +557,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dv = FP8 ? smem_desc(v_addr, 16, 8 * 128, 2u)
                                     : smem_desc(v_addr, C::kAtomBytes, C::kSBO, C::kLayout);
             // S_i = Q_i K^T: both operands K-major, 32 bytes of the head dim per step
+            // Descriptor offsets never carry out of the low word (shared addresses < 256 KB): the
+            // low words are advanced with 32-bit adds and the high words are constants.
+            const uint32_t dq_lo = static_cast<uint32_t>(dq), dq_hi = static_cast<uint32_t>(dq >> 32);
+            const uint32_t dk_lo = static_cast<uint32_t>(dk), dk_hi = static_cast<uint32_t>(dk >> 32);
+            const uint32_t dv_lo = static_cast<uint32_t>(dv), dv_hi = static_cast<uint32_t>(dv >> 32);
+            auto desc = [](uint32_t lo, uint32_t hi) {
+                uint64_t d;
+                asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+                return d;
+            };
+            const bool leader = elect_one();     // the lane that issues (elected once)
             auto issue_s = [&](int i, uint32_t kst) {
-                const uint64_t qb = dq + ((i * C::kTileBytes) >> 4);
-                const uint64_t kb = dk + ((kst * C::kTileBytes) >> 4);
-                if (elect_one()) {
+                const uint32_t qb = dq_lo + ((i * C::kTileBytes) >> 4);
+                const uint32_t kb = dk_lo + ((kst * C::kTileBytes) >> 4);
+                if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < D / C::kK; ++kk) {
                         const uint32_t off = C::kstep(kk);
-                        if constexpr (FP8) mma_ss_f8(tmem + kColS[i], qb + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
-                        else mma_ss(tmem + kColS[i], qb + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
+                        if constexpr (FP8)
+                            mma_ss_f8(tmem + kColS[i], desc(qb + off, dq_hi), desc(kb + off, dk_hi), idesc_s, kk > 0 ? 1u : 0u);
+                        else
+                            mma_ss(tmem + kColS[i], desc(qb + off, dq_hi), desc(kb + off, dk_hi), idesc_s, kk > 0 ? 1u : 0u);
                     }
                 }
-                __syncwarp();
             };
             // O_i += P_i V: P from tensor memory (8 columns per step), kK keys per step of V: kK rows
             // of the N(=d)-major 16-bit V, or 32 bytes along each row of the e4m3 V^T
             auto issue_pv = [&](int i, uint32_t vst, bool acc) {
-                const uint64_t vb = dv + ((vst * C::kTileBytes) >> 4);
-                if (elect_one()) {
+                const uint32_t vb = dv_lo + ((vst * C::kTileBytes) >> 4);
+                if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < kBlockN / C::kK; ++kk) {
-                        const uint64_t vk = vb + (FP8 ? ((kk * 32) >> 4) : ((kk * C::kK * C::kRowBytes) >> 4));
+                        const uint64_t vk = desc(vb + (FP8 ? ((kk * 32) >> 4) : ((kk * C::kK * C::kRowBytes) >> 4)), dv_hi);
                         if constexpr (FP8)
                             mma_ts_f8(tmem + kColO[i], tmem + kColP[i] + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
                         else
                             mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
                     }
                 }
-                __syncwarp();
             };
             auto commit = [&](uint64_t* bar) {
-                if (elect_one()) mma_commit(bar);
-                __syncwarp();
+                if (leader) mma_commit(bar);
             };
             uint32_t kc = 0, vc = 0, uit = 0;
             uint32_t pv_cnt[2] = {0, 0}, sf_cnt[2] = {0, 0};
