@@ -508,19 +508,6 @@ attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const att
         if (sms > 0 && kv_bytes > static_cast<double>(l2_bytes())) g = (sms + p.num_q_pairs - 1) / p.num_q_pairs;
         p.head_group = g < 1 ? 1 : (g > B * H ? static_cast<int>(B * H) : g);
     }
-    // a bias shared over the batch whose tiles of a unit all fit the staging slots (the
-    // Evoformer row attention, N <= 256 at d = 32): blocked, head-major unit order, so that a
-    // CTA copies a head's bias tiles once instead of once per unit (units are equal without
-    // causal masking, so the blocked order balances as well as the interleaved one)
-    p.blocked = 0;
-    if (bias != nullptr && bias->ndim == 3 && !causal && d <= 64 && (mods == nullptr || (mods->alibi_slopes == nullptr && mods->softcap <= 0.f && mods->window_left < 0))) {
-        const int slots = d == 32 ? attn::BiasCfg<32, true>::kStages : attn::BiasCfg<64, true>::kStages;
-        const int sms = sm_count();
-        if (sms > 0 && p.n_kv_tiles <= slots) {
-            const int grid = p.num_units < sms ? p.num_units : sms;
-            p.blocked = (p.num_units + grid - 1) / grid;
-        }
-    }
     if (bias != nullptr) {
         p.bias = bias->data;
         if (bias->ndim == 3) {

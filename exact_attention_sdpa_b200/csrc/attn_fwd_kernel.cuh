@@ -95,10 +95,6 @@ struct FwdParams {
     unsigned int* status;
     int inject_stall;          // test hook: the MMA warp first waits on a barrier nothing arrives on
     float v_scale;             // e4m3 inputs: the value tensor's scale (the query and key scales are in scale)
-    // blocked unit order (> 0: units per CTA): CTA b takes units [b * blocked, (b + 1) * blocked),
-    // decoded head-major, so that consecutive units of a CTA share a head and hence a bias
-    // shared over the batch, which then stays in its staging slots (see load_bias)
-    int blocked;
     // ragged batch in one launch (n_seq > 0; B = 1 and the tensors are packed [1, H, T, d] views):
     // sequence s owns query rows seq_q0[s] .. + seq_nq[s] and key rows seq_k0[s] .. + seq_nk[s],
     // and units seq_units[s] .. seq_units[s + 1] (its query pairs x H, heaviest pairs first)
@@ -293,9 +289,8 @@ struct Unit {
 // [k G, (k+1) G) of the heaviest-first order, G = gridDim.x, forwards for even k and
 // backwards for odd k: the CTA that drew the heaviest unit of one wave draws the
 // lightest of the next, which evens out the per-CTA totals of causal workloads.
-__device__ __forceinline__ int unit_at(int k, const FwdParams& p) {
+__device__ __forceinline__ int unit_at(int k) {
     const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-    if (p.blocked > 0) return k < p.blocked ? min(b * p.blocked + k, p.num_units) : p.num_units;
     return k * G + ((k & 1) ? (G - 1 - b) : b);
 }
 
@@ -320,17 +315,6 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
         U.h = r % p.H;
         U.b = 0;
         U.bh = U.h;
-    } else if (p.blocked > 0) {
-        // head-major: a CTA's consecutive units share a head (query pairs, then batches, then heads)
-        U.qp = u % p.num_q_pairs;
-        const int rest = u / p.num_q_pairs;
-        U.b = rest % p.B;
-        U.h = rest / p.B;
-        U.bh = U.b * p.H + U.h;
-        U.N = p.N;
-        U.Nk = p.Nk;
-        U.q_base = 0;
-        U.k_base = 0;
     } else {
         // Units are taken in groups of `head_group` heads; inside a group the heaviest query
         // pairs come first (causal load balance).  With head_group = B*H (the default) this is
@@ -482,37 +466,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++qc[i];
             };
             uint32_t bc[2] = {0, 0};            // bias tiles loaded per query tile
-            // what each bias slot holds (batch, head, first row, first key; -1: nothing yet): a
-            // slot that already holds the tile is not copied again, only its full barrier is
-            // arrived on (a bias shared over the batch, blocked unit order: once per CTA and head)
-            int slot_tag[2][BC::kStages > 0 ? BC::kStages : 1][4];
-            for (int i = 0; i < 2; ++i)
-                for (int s2 = 0; s2 < BC::kStages; ++s2) slot_tag[i][s2][0] = -1;
             auto load_bias = [&](int i, int j, const Unit& U) {
                 const uint32_t st = bc[i] % BC::kStages;
                 if (bc[i] >= BC::kStages &&
                     !WU(&sh.bias_empty[i][st], ((bc[i] / BC::kStages) - 1) & 1))
                     return;
-                const int bb = p.bias_sb != 0 ? U.b : 0;
-                const int row0 = U.q0 + i * kBlockM, key0 = (U.kv_lo + j) * kBlockN;
-                int* tag = slot_tag[i][st];
-                const bool held = tag[0] == bb && tag[1] == U.h && tag[2] == row0 && tag[3] == key0;
                 if (elect_one()) {
-                    if (held) {
-                        mbar_arrive(&sh.bias_full[i][st]);
-                    } else {
-                        mbar_arrive_expect_tx(&sh.bias_full[i][st], BC::kTileBytes);
-                        uint8_t* dst = sBias + (i * BC::kStages + st) * BC::kTileBytes;
-                        for (int half = 0; half < 2; ++half)
-                            tma_load_4d(dst + half * BC::kBoxBytes, &tm_bias, &sh.bias_full[i][st],
-                                        key0 + half * 64, row0, U.h, bb, pol_kv);
-                    }
+                    mbar_arrive_expect_tx(&sh.bias_full[i][st], BC::kTileBytes);
+                    uint8_t* dst = sBias + (i * BC::kStages + st) * BC::kTileBytes;
+                    const int bb = p.bias_sb != 0 ? U.b : 0;
+                    for (int half = 0; half < 2; ++half)
+                        tma_load_4d(dst + half * BC::kBoxBytes, &tm_bias, &sh.bias_full[i][st],
+                                    (U.kv_lo + j) * kBlockN + half * 64, U.q0 + i * kBlockM, U.h, bb, pol_kv);
                 }
                 __syncwarp();
-                tag[0] = bb;
-                tag[1] = U.h;
-                tag[2] = row0;
-                tag[3] = key0;
                 ++bc[i];
             };
             auto load_kv = [&](uint64_t* full, uint64_t* empty, uint8_t* ring, const CUtensorMap* map, uint32_t& cnt,
@@ -536,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 ++cnt;
             };
-            for (int k = 0, u = unit_at(0, p); ok && u < p.num_units; u = unit_at(++k, p)) {
+            for (int k = 0, u = unit_at(0); ok && u < p.num_units; u = unit_at(++k)) {
                 const Unit U = decode_unit<CAUSAL, MODS>(u, p);
                 // the unit's first bias tiles go first: their stages free up as soon as the
                 // softmax has read the previous unit's first tiles, long before the Q slots do
@@ -656,9 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // after both tiles' last PVs, so tile 0's softmax restarts one PV group earlier.
             // Issued after that PV, S_i(0) needs no further ordering: its commit covers the PV.
             bool early[2] = {false, false};
-            for (int u = unit_at(0, p); ok && u < p.num_units; u = unit_at(++uit, p)) {
+            for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
                 const Unit U = decode_unit<CAUSAL, MODS>(u, p);
-                const int u_next = unit_at(uit + 1, p);
+                const int u_next = unit_at(uit + 1);
                 int nkv_next[2] = {0, 0};      // 0: no next unit
                 if (C::kSeparateP && u_next < p.num_units) {
                     const Unit Un = decode_unit<CAUSAL, MODS>(u_next, p);
@@ -784,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool fast = !HAS_BIAS && scale_log2 > 0.f && (!MODS || (p.alibi == nullptr && p.softcap <= 0.f));
         uint32_t s_cnt = 0, od_cnt = 0, bcnt = 0, uit = 0;
         bool ok = true;
-        for (int u = unit_at(0, p); ok && u < p.num_units; u = unit_at(++uit, p)) {
+        for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
             const Unit U = decode_unit<CAUSAL, MODS>(u, p);
             const int nkv = i ? U.nkv1 : U.nkv0;
             const int row = U.q0 + i * kBlockM + t;
@@ -1037,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return ok;
         };
         const bool has_next_unit_pv_arrival = !C::kInlineRescale;
-        for (int u = unit_at(0, p); ok && u < p.num_units; u = unit_at(++uit, p)) {
+        for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
             const Unit U = decode_unit<CAUSAL, MODS>(u, p);
             if constexpr (!C::kInlineRescale) {
                 // d = 128, the correction: O_i *= alpha(j) between PV_i(j-1) and PV_i(j) (only when
@@ -1082,7 +1049,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // its last chunk is in registers (at d = 128 together with the next unit's first
             // pv_ready arrival: iteration 0 needs no rescale), so the next unit's PV_i(0) does not
             // wait for the gate arithmetic and the global stores.
-            const bool has_next = has_next_unit_pv_arrival && unit_at(uit + 1, p) < p.num_units;
+            const bool has_next = has_next_unit_pv_arrival && unit_at(uit + 1) < p.num_units;
             for (int i = 0; i < 2; ++i) {
                 const int row = U.q0 + i * kBlockM + t;
                 const bool row_ok = row < U.N;

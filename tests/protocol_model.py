@@ -104,7 +104,6 @@ class Config:
     plant: str = ""               # a protocol mistake planted on purpose (tests of the checker)
     timeout: tuple = ()           # (role, n): that role's n-th bounded wait gives up (abort path)
     tma_weight: float = 1.0       # relative chance that a pending TMA load completes next (< 1: slow loads)
-    bias_reuse: bool = False      # every unit has the same bias tiles: a slot that holds its tile is not copied
 
 
 def random_units(rng: random.Random, causal: bool, n_units: int, max_tiles: int = 5) -> list:
@@ -213,8 +212,6 @@ def producer(st: State):
         yield Tma(f"{kind} tile {n}", run, full[s_])
         cnt[kind] += 1
 
-    held = {}                      # (tile, slot) -> the key tile it holds (bias_reuse)
-
     def load_bias(i, j, k):
         s_ = bc[i] % BS
         if bc[i] >= BS and not (yield from WU(st.bias_empty[i][s_], ((bc[i] // BS) - 1) & 1, bc[i] // BS - 1)):
@@ -222,13 +219,7 @@ def producer(st: State):
 
         def run(s, i=i, s_=s_, j=j, k=k):
             s.sBias[i][s_] = (k, j)
-        if cfg.bias_reuse and held.get((i, s_)) == j:
-            # the slot already holds this (identical) tile: only its full barrier is arrived on
-            yield Do(f"bias{i} ({k},{j}) held", run)
-            yield Arrive(st.bias_full[i][s_], 1)
-        else:
-            yield Tma(f"bias{i} ({k},{j})", run, st.bias_full[i][s_])
-        held[(i, s_)] = j
+        yield Tma(f"bias{i} ({k},{j})", run, st.bias_full[i][s_])
         bc[i] += 1
 
     for k, (n0, n1) in enumerate(cfg.units):

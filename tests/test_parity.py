@@ -223,13 +223,3 @@ def test_rectangular_q_and_kv(N, Nk, causal, d, dtype, bias, gate):
         dead = N - Nk
         assert torch.all(o[:, :, :dead] == 0)
         assert torch.all(torch.isneginf(lse[:, :, :dead]))
-
-
-@pytest.mark.parametrize("B,H,N,d", [(64, 5, 100, 64), (90, 7, 256, 32), (333, 2, 129, 32)])
-def test_shared_bias_blocked_order(B, H, N, d):
-    """A pair bias shared over the batch, without causal masking, whose tiles fit the staging
-    slots: each CTA takes a run of consecutive head-major units and copies a head's bias tiles
-    once (later units only re-arm the slots).  Several units per CTA, heads changing inside a
-    CTA's run, a ragged last tile; every row compared."""
-    w = Workload("blk", B=B, H=H, N=N, d=d, dtype="bf16", causal=False, seed=400 + N, bias=True, gate=(d == 32))
-    _full_check(w)

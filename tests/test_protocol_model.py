@@ -46,17 +46,6 @@ def test_protocol_holds_over_long_unit_sequences(sep):
         pm.run(cfg, seed=rep)
 
 
-def test_bias_slots_reused_across_units():
-    # a bias shared over the batch in the blocked unit order: every unit's bias tiles are the
-    # same, and a slot that holds its tile is only arrived on, not copied again
-    for rep in range(150):
-        rng = random.Random(900 + rep)
-        n = rng.randint(1, 2)
-        cfg = pm.Config(separate_p=True, causal=False, stages=4, bias_stages=2, bias_reuse=True,
-                        units=[(n, n)] * rng.randint(1, 6), tma_weight=0.03 if rep % 2 else 1.0)
-        pm.run(cfg, seed=rep)
-
-
 def test_single_tile_units_back_to_back():
     # units with one key tile each: S_i(0) of the next unit, Q release and the statistics
     # double buffer are exercised on every unit

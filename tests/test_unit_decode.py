@@ -38,12 +38,6 @@ def decode(u, p):
         U["qp"] = nqp - 1 - r // p["H"]
         U["h"] = r % p["H"]
         U["seq"] = lo
-    elif p.get("blocked", 0) > 0:
-        # head-major: query pairs, then batches, then heads
-        U["qp"] = u % p["num_q_pairs"]
-        rest = u // p["num_q_pairs"]
-        U["seq"], U["h"] = rest % p["B"], rest // p["B"]
-        U["N"], U["Nk"] = p["N"], p["Nk"]
     else:
         BH, G = p["B"] * p["H"], p["head_group"]
         per = G * p["num_q_pairs"]
@@ -105,33 +99,10 @@ def check_units(p, problems):
     assert seen == want
 
 
-def dense_params(B, H, N, Nk, causal, window=-1, head_group=None, blocked=0):
+def dense_params(B, H, N, Nk, causal, window=-1, head_group=None):
     nqp = (N + ROWS_PER_UNIT - 1) // ROWS_PER_UNIT
     return {"n_seq": 0, "B": B, "H": H, "N": N, "Nk": Nk, "num_q_pairs": nqp, "num_units": nqp * B * H,
-            "head_group": head_group or B * H, "causal": causal, "window_left": window, "mods": window >= 0,
-            "blocked": blocked}
-
-
-def unit_at(k, b, G, p):
-    """Mirror of unit_at: the k-th unit of CTA b of a grid of G."""
-    if p.get("blocked", 0) > 0:
-        return min(b * p["blocked"] + k, p["num_units"]) if k < p["blocked"] else p["num_units"]
-    return k * G + ((G - 1 - b) if k & 1 else b)
-
-
-def cta_units(p, G):
-    """The unit sequence of every CTA, as the persistent kernel walks it."""
-    out = []
-    for b in range(G):
-        seq, k = [], 0
-        while True:
-            u = unit_at(k, b, G, p)
-            if u >= p["num_units"]:
-                break
-            seq.append(u)
-            k += 1
-        out.append(seq)
-    return out
+            "head_group": head_group or B * H, "causal": causal, "window_left": window, "mods": window >= 0}
 
 
 @pytest.mark.parametrize("seed", range(40))
@@ -145,27 +116,6 @@ def test_dense_problems_with_windows(seed):
     hg = rng.randint(1, B * H)
     problems = {b: (N, Nk) for b in range(B)}
     check_units(dense_params(B, H, N, Nk, causal, window, hg), problems)
-
-
-@pytest.mark.parametrize("seed", range(20))
-def test_every_unit_runs_once_on_some_cta(seed):
-    """Both unit orders hand every unit to exactly one CTA; the blocked order (a bias shared over
-    the batch) gives each CTA a run of consecutive units, mostly of one head."""
-    rng = random.Random(500 + seed)
-    B, H, N = rng.randint(1, 40), rng.randint(1, 9), rng.randint(1, 700)
-    blocked_mode = seed % 2 == 0
-    p = dense_params(B, H, N, N, causal=not blocked_mode)
-    G = min(p["num_units"], rng.choice([1, 7, 148]))
-    if blocked_mode:
-        p["blocked"] = (p["num_units"] + G - 1) // G
-    seqs = cta_units(p, G)
-    flat = sorted(u for s in seqs for u in s)
-    assert flat == list(range(p["num_units"]))
-    if blocked_mode:
-        check_units(p, {b: (N, N) for b in range(B)})
-        for s in seqs:
-            heads = [decode(u, p)["h"] for u in s]
-            assert heads == sorted(heads)            # a CTA changes head at most a few times, in order
 
 
 def varlen_params(lengths, H, causal):
