@@ -399,12 +399,12 @@ cudaError_t launch_bwd_tc_t(const BwdMaps& m, const attn::bwdtc::Params& p, cuda
     constexpr int s1 = DkdvCfg<D>::kDynBytes;
     static std::atomic<uint64_t> set1{0}, set2{0};
     if ((e = smem_limit_once(k1, s1, set1)) != cudaSuccess) return e;
-    k1<<<dim3((p.Nk + 127) / 128, p.B * p.H), kThreads, s1, stream>>>(m.q64, m.k128, m.v128, m.do64, p);
+    k1<<<dim3((p.Nk + 127) / 128, p.B * p.H), kThreadsPP, s1, stream>>>(m.q64, m.k128, m.v128, m.do64, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     auto k2 = bwd_dq_kernel<T, D, CAUSAL, MODS>;
     constexpr int s2 = DqCfg<D>::kDynBytes;
     if ((e = smem_limit_once(k2, s2, set2)) != cudaSuccess) return e;
-    k2<<<dim3((p.N + 127) / 128, p.B * p.H), kThreads, s2, stream>>>(m.q128, m.k64, m.v64, m.do128, p);
+    k2<<<dim3((p.N + 127) / 128, p.B * p.H), kThreadsPP, s2, stream>>>(m.q128, m.k64, m.v64, m.do128, p);
     return cudaGetLastError();
 }
 

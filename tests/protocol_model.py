@@ -659,8 +659,10 @@ def run(cfg: Config, seed: int, make_roles=kernel_roles, state_cls=State, max_st
             if info is not None:
                 info["aborted"] = st.abort
             return steps
-        if cfg.tma_weight != 1.0:
-            weights = [cfg.tma_weight if c[0] == "tma" else 1.0 for c in choices]
+        slow = getattr(cfg, "slow_roles", ())     # roles that move rarely (late warps)
+        if cfg.tma_weight != 1.0 or slow:
+            weights = [cfg.tma_weight if c[0] == "tma" else (0.02 if c[0] == "role" and c[1] in slow else 1.0)
+                       for c in choices]
             kind, key = rng.choices(choices, weights)[0]
         else:
             kind, key = rng.choice(choices)
