@@ -25,6 +25,10 @@ CASES = [  # B, H, N, Nk, d, causal, dtype
     (1, 4, 257, 257, 128, False, "fp16"),
     (1, 1, 1, 500, 64, True, "bf16"),
     (2, 2, 384, 384, 32, False, "bf16"),
+    # fewer column blocks than TMEM column sets: dK/dV sees 2 query blocks and dQ 3 key blocks
+    # (three sets at d=64), then 3 and 2 at d=128 (two sets)
+    (1, 2, 128, 192, 64, False, "fp16"),
+    (1, 2, 192, 128, 128, False, "bf16"),
 ]
 
 
