@@ -250,7 +250,8 @@ __device__ __forceinline__ bool group_sync_and(uint32_t id, bool pred) {
 // Shared-memory operand ring and the barriers of one CTA.
 template <int ST>
 struct PipeBars {
-    uint64_t row_full;             // the CTA's own 128-row operands (K, V or Q, dO)
+    uint64_t row_full;             // the CTA's own 128-row operands (K, V or Q, dO) in shared memory
+    uint64_t row_tmem;             // dQ: Q and dO copied into tensor memory (both groups, 256 arrivals)
     uint64_t full[ST], empty[ST];  // column-block operand stages
     uint64_t s_full[3];            // column set c holds its block's two products (issuer commit)
     uint64_t p_ready[3];           // set c holds its block's 16-bit operands (the group's 128
@@ -262,6 +263,7 @@ struct PipeBars {
 template <int ST>
 __device__ __forceinline__ void init_pipe(PipeBars<ST>& br) {
     sm100::mbar_init(&br.row_full, 1);
+    sm100::mbar_init(&br.row_tmem, 256);
     for (int s = 0; s < ST; ++s) {
         sm100::mbar_init(&br.full[s], 1);
         sm100::mbar_init(&br.empty[s], 1);
@@ -297,16 +299,17 @@ __device__ __forceinline__ void produce(PipeBars<ST>& br, int nit, int* abort_p,
 }
 
 // Tensor-core issuer: the whole warp runs the loop, so that its waits and descriptor arithmetic
-// are warp-uniform, and the elected lane `leader` issues.  products(s, col) fills the column set
+// are warp-uniform, and the elected lane `leader` issues.  It starts once `row_ready` completed
+// (the row block's operands are in place).  products(s, col) fills the column set
 // at `col` from stage s, accumulate(m, s, col) consumes it; the final commit on acc_done covers
 // every product, and the warp waits for it before returning (the CTA frees tensor memory after).
 template <int ST, int SETS, typename Products, typename Accumulate>
-__device__ __forceinline__ void issue(PipeBars<ST>& br, int nit, int* abort_p, const Params& p, bool leader,
-                                      Products products, Accumulate accumulate) {
+__device__ __forceinline__ void issue(PipeBars<ST>& br, uint64_t* row_ready, int nit, int* abort_p, const Params& p,
+                                      bool leader, Products products, Accumulate accumulate) {
     auto W = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_p, p));
     };
-    bool ok = W(&br.row_full, 0);
+    bool ok = W(row_ready, 0);        // the row block's operands (row_full, or row_tmem for dQ)
     auto prod = [&](int m) -> bool {
         if (!W(&br.full[m % ST], (m / ST) & 1)) return false;
         sm100::tc_fence_after();
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
                 const uint64_t qn = TQ::desc_n(sQ), don = TQ::desc_n(sdO);
                 const bool leader = elect_one();
                 issue<ST, C::kSets>(
-                    br, nit, abort_p, p, leader,
+                    br, &br.row_full, nit, abort_p, p, leader,
                     [&](int s, uint32_t col) {             // S^T = K Q^T, dP^T = V dO^T
                         const uint32_t so = (s * TQ::kBytes) >> 4;
                         if (leader) {
@@ -608,7 +611,10 @@ struct DqCfg {
     static constexpr int kSets = (kStages >= 5) ? 3 : 2;
     static constexpr uint32_t kCols = 512u;
     static constexpr uint32_t kColDQ = 128 * kSets;              // after the sets
-    static_assert(kColDQ + D <= kCols, "tensor memory budget");
+    // Q and dO, 16-bit pairs per column: the A operands of the products (TS form, whose only
+    // shared-memory operand is the key block: SS products at N = 64 are bound by their operand reads)
+    static constexpr uint32_t kColQ = kColDQ + D, kColDO = kColQ + D / 2;
+    static_assert(kColDO + D / 2 <= kCols, "tensor memory budget");
     static constexpr int kOffQ = 0, kOffDO = TQ::kBytes, kOffK = 2 * TQ::kBytes;
     static constexpr int kOffV = kOffK + kStages * TK::kBytes;
     static constexpr int kBytes = kOffV + kStages * TK::kBytes;
@@ -692,22 +698,21 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
             if (nit > 0) {
                 constexpr uint32_t idesc_s = instr_desc_f16(kBF16, 128, 64, false);
                 constexpr uint32_t idesc_o = instr_desc_f16(kBF16, 128, D, true);
-                const uint64_t dq_ = TQ::desc_k(sQ), ddo = TQ::desc_k(sdO);
                 const uint64_t dk_ = TK::desc_k(sK), dv_ = TK::desc_k(sV);     // stage 0
                 const uint64_t kn = TK::desc_n(sK);
                 const bool leader = elect_one();
                 issue<ST, C::kSets>(
-                    br, nit, abort_p, p, leader,
-                    [&](int s, uint32_t col) {             // S = Q K^T, dP = dO V^T
+                    br, &br.row_tmem, nit, abort_p, p, leader,
+                    [&](int s, uint32_t col) {             // S = Q K^T, dP = dO V^T (Q, dO in TMEM)
                         const uint32_t so = (s * TK::kBytes) >> 4;
                         if (leader) {
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(tmem + col, desc_at(lo32(dq_) + TQ::kstep(kk), hi32(dq_)),
+                                mma_ts(tmem + col, tmem + C::kColQ + kk * 8,
                                        desc_at(lo32(dk_) + so + TK::kstep(kk), hi32(dk_)), idesc_s, kk > 0 ? 1u : 0u);
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(tmem + col + 64, desc_at(lo32(ddo) + TQ::kstep(kk), hi32(ddo)),
+                                mma_ts(tmem + col + 64, tmem + C::kColDO + kk * 8,
                                        desc_at(lo32(dv_) + so + TK::kstep(kk), hi32(dv_)), idesc_s, kk > 0 ? 1u : 0u);
                         }
                     },
@@ -740,8 +745,42 @@ __global__ void __launch_bounds__(kThreadsPP, 1)
             nlse2 = -p.lse[static_cast<int64_t>(bh) * p.N + qi] * kLog2e;
             ndrow = -*reinterpret_cast<const float*>(dqrow);
         }
-        const float slope = (MODS && p.alibi != nullptr) ? p.alibi[h] : 0.f;
         bool ok = true;
+        if (nit > 0) {
+            // this thread's row of Q (group 0) or dO (group 1) from the TMA-written tile (128- or,
+            // at d = 32, 64-byte swizzle) into tensor memory, the A operand of the products
+            ok = __all_sync(0xffffffffu, wait_bar(&br.row_full, 0, abort_p, p));
+            if (ok) {
+                tc_fence_after();
+                const uint8_t* row = (g == 0 ? sQ : sdO) + tw * TQ::kRowBytes;
+                constexpr int kChunks = TQ::kRowBytes / 16;            // 16-byte chunks per atom row
+                const int swz = (kChunks == 8) ? (tw & 7) : ((tw >> 1) & 3);
+                uint32_t w[D / 2];
+#pragma unroll
+                for (int a = 0; a < TQ::kNumAtoms; ++a)
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(row + a * TQ::kAtomBytes + ((c ^ swz) << 4));
+                        const int o = (a * kChunks + c) * 4;
+                        w[o] = v.x;
+                        w[o + 1] = v.y;
+                        w[o + 2] = v.z;
+                        w[o + 3] = v.w;
+                    }
+                const uint32_t dst = tmem + lane_off + (g == 0 ? C::kColQ : C::kColDO);
+                if constexpr (D == 32) {
+                    tmem_st16(dst, w);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c)
+                        tmem_st32(dst + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&w[c * 32]));
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&br.row_tmem);
+            }
+        }
+        const float slope = (MODS && p.alibi != nullptr) ? p.alibi[h] : 0.f;
         for (int m = g; m < nit; m += 2) {
             ok = group_sync_and(1 + g, ok);
             if (!ok) break;

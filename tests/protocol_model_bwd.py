@@ -17,6 +17,11 @@ protocol over a CTA's 128-row block and its nit column blocks:
     the bounded acc_done wait (dQ: group g stores 32-column chunks g, g + 2, ...; chunk 0 holds
     the D value the dQ groups read before their first block).
 
+dQ only: the products take Q and dO from tensor memory (TS form).  Each group warp waits for
+the row block's TMA load (row_full), copies its rows of Q (group 0) or dO (group 1) from
+shared into tensor memory and arrives on row_tmem (256 arrivals); the issuer waits for
+row_tmem instead of row_full.
+
 Version tags: the products in a column set are ("prod", m) and, once a warp stored its
 operands, ("ops", m); the accumulators count the blocks accumulated; a stage holds the column
 block loaded into it; the lse/D buffer holds the block it was written for; the dQ row's chunk
@@ -50,6 +55,7 @@ class BwdState:
         self.cfg = cfg
         B, ST = Barrier, cfg.stages
         self.row_full = B("row_full", 1)
+        self.row_tmem = B("row_tmem", 128 * 2)
         self.full = [B(f"full{s}", 1) for s in range(ST)]
         self.empty = [B(f"empty{s}", 1) for s in range(ST)]
         self.s_full = [B(f"s_full{c}", 1) for c in range(cfg.sets)]
@@ -61,6 +67,7 @@ class BwdState:
         self.votes = [dict(), dict()]          # [group][barrier use] -> AND of the warps' flags
         # buffers
         self.s_row = None
+        self.t_row = [[None] * GROUP_WARPS for _ in range(2)]    # dQ: [group][lane quarter] of Q / dO
         self.s_col = [None] * ST
         self.t_set = [[None] * GROUP_WARPS for _ in range(cfg.sets)]   # [column set][lane quarter]
         self.acc = 0
@@ -112,7 +119,12 @@ def issuer(st: BwdState):
             s_, c = m % ST, m % SETS
 
             def run_(s, m=m, s_=s_, c=c):
-                s.expect("row operands", s.s_row, "row")
+                if s.cfg.kind == "dq":
+                    for g in range(2):
+                        for q in range(GROUP_WARPS):
+                            s.expect(f"row operand {g} in tensor memory, quarter {q}", s.t_row[g][q], "row")
+                else:
+                    s.expect("row operands", s.s_row, "row")
                 s.expect(f"stage {s_} for products({m})", s.s_col[s_], m)
                 for q in range(GROUP_WARPS):
                     s.t_set[c][q] = ("prod", m)
@@ -135,7 +147,12 @@ def issuer(st: BwdState):
             yield Issue("mma", f"accumulate({m})", run_)
             yield Commit("mma", st.empty[s_])
 
-        ok = yield Wait(st.row_full, 0, 0)
+        if cfg.kind == "dq" and cfg.plant != "mma_skips_row_tmem":
+            ok = yield Wait(st.row_tmem, 0, 0)
+        elif cfg.kind == "dq":
+            ok = True
+        else:
+            ok = yield Wait(st.row_full, 0, 0)
         m = 0
         while ok and m < SETS and m < nit:
             ok = yield from products(m)
@@ -172,6 +189,16 @@ def group_warp(st: BwdState, g: int, q: int):
             s.expect(f"D of quarter {q}", s.dq_chunk0[q], "D")
         yield Do(f"read D (quarter {q})", read_d)
     ok = True
+    if not dkdv and nit > 0:
+        # the row block's operand into tensor memory (TS products)
+        if cfg.plant != "copy_without_row_full":
+            ok = yield Wait(st.row_full, 0, 0)
+        if ok:
+            def copy(s, q=q):
+                s.expect(f"row block in shared memory (quarter {q})", s.s_row, "row")
+                s.t_row[g][q] = "row"
+            yield Do(f"copy row operand {g} (quarter {q})", copy)
+            yield Arrive(st.row_tmem, 32)
     it = 0
     for m in range(g, nit, 2):
         buf = 0 if cfg.plant == "lse_single_buffer" else it & 1

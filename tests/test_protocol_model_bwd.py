@@ -34,8 +34,9 @@ def test_bwd_timeout_at_any_wait_exits_cleanly(kind, sets):
 
 PLANTS = [("empty_parity", "dkdv", 7, 2), ("prod_before_acc", "dkdv", 5, 2), ("prod_before_acc", "dq", 5, 3),
           ("no_s_full_wait", "dq", 4, 2), ("no_s_full_wait", "dkdv", 6, 3), ("lse_single_buffer", "dkdv", 6, 2),
-          ("dq_reads_d_without_block", "dq", 1, 3), ("p_ready_per_group", "dkdv", 8, 3),
-          ("p_ready_per_group", "dq", 8, 3)]
+          ("p_ready_per_group", "dkdv", 8, 3),
+          ("p_ready_per_group", "dq", 8, 3), ("mma_skips_row_tmem", "dq", 4, 3),
+          ("copy_without_row_full", "dq", 4, 3)]
 
 
 SLOW = [(), ("grp1.0", "grp1.3"), ("grp0.2", "grp1.1"), ("mma",)]
@@ -67,10 +68,20 @@ def test_bwd_model_barriers_match_the_kernel_source():
     src = open(os.path.join(os.path.dirname(__file__), "..", "exact_attention_sdpa_b200", "csrc",
                             "attn_bwd_tc.cuh")).read()
     inits = dict(re.findall(r"mbar_init\(&br\.(\w+)(?:\[\w+\])?, (\d+)\)", src))
-    assert inits == {"row_full": "1", "full": "1", "empty": "1", "s_full": "1", "p_ready": "128", "acc_done": "1"}
+    assert inits == {"row_full": "1", "row_tmem": "256", "full": "1", "empty": "1", "s_full": "1", "p_ready": "128",
+                     "acc_done": "1"}
     assert "bar.red.and.pred q, %2, 128, p;" in src
     assert re.search(r"constexpr int kMmaWarp = 8, kTmaWarp = 9;", src)
     # column sets: 3 for dQ and, where tensor memory holds them beside dK and dV, for dK/dV
-    assert "static constexpr int kSets = (3 * 128 + 2 * D <= 512) ? 3 : 2;" in src
-    assert "static constexpr int kSets = 3;" in src
+    assert "static constexpr int kSets = (3 * 128 + 2 * D <= 512 && kStages >= 5) ? 3 : 2;" in src
+    assert "static constexpr int kSets = (kStages >= 5) ? 3 : 2;" in src
     assert "        sm100::mbar_init(&br.s_full[c], 1);\n        sm100::mbar_init(&br.p_ready[c], 128);" in src
+
+
+def test_dq_d_read_guard_is_a_second_guard():
+    """A dQ group without a block reading D would race group 0's store over chunk 0 -- but every
+    group arrives on row_tmem (after its D read) before the first product can run, so that
+    arrival orders the read as well; the kernel's `nit > g` guard is kept as a second one."""
+    for seed in range(300):
+        run_bwd(BwdConfig(kind="dq", nit=1, stages=4, sets=3, plant="dq_reads_d_without_block",
+                          slow_roles=SLOW[seed % len(SLOW)]), seed)
