@@ -203,6 +203,61 @@ bool encode_bias_map(CUtensorMap* map, const attn_tensor_t* b) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Encoded tensor maps, cached per (base pointer, dtype, rank, shape, strides, box rows, map
+// kind): a map depends on nothing else, so a call on buffers seen before skips the driver's
+// encode.  64 entries replaced round-robin; lookups and inserts under one mutex.
+enum MapKind { kMapQkv = 0, kMapE4m3 = 1, kMapE4m3Vt = 2, kMapBias = 3 };
+struct MapKey {
+    const void* data;
+    int64_t shape[4], stride[4];
+    int32_t dtype, ndim, kind;
+    uint32_t rows;
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+std::mutex g_map_mu;
+MapEntry g_maps[64];
+unsigned g_map_next = 0;
+
+bool encode_map(MapKind kind, CUtensorMap* map, const attn_tensor_t* t, unsigned rows) {
+    MapKey k;
+    std::memset(&k, 0, sizeof(k));            // padding included: keys compare with memcmp
+    k.data = t->data;
+    for (int i = 0; i < t->ndim && i < 4; ++i) {
+        k.shape[i] = t->shape[i];
+        k.stride[i] = t->stride[i];
+    }
+    k.dtype = static_cast<int32_t>(t->dtype);
+    k.ndim = t->ndim;
+    k.kind = kind;
+    k.rows = rows;
+    {
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        for (const MapEntry& e : g_maps)
+            if (e.used && std::memcmp(&e.key, &k, sizeof(k)) == 0) {
+                *map = e.map;
+                return true;
+            }
+    }
+    bool ok = false;
+    switch (kind) {
+        case kMapQkv: ok = encode_qkv_map(map, t, rows); break;
+        case kMapE4m3: ok = encode_e4m3_map(map, t); break;
+        case kMapE4m3Vt: ok = encode_e4m3_vt_map(map, t); break;
+        case kMapBias: ok = encode_bias_map(map, t); break;
+    }
+    if (!ok) return false;
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    MapEntry& e = g_maps[g_map_next++ % 64];
+    e.key = k;
+    e.map = *map;
+    e.used = true;
+    return true;
+}
+
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
@@ -478,10 +533,11 @@ attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const att
     // ---- launch
     Maps maps;
     std::memset(&maps, 0, sizeof(maps));
-    if (!encode_qkv_map(&maps.q, q) || !encode_qkv_map(&maps.k, k) || !encode_qkv_map(&maps.v, v))
+    if (!encode_map(kMapQkv, &maps.q, q, 128) || !encode_map(kMapQkv, &maps.k, k, 128) ||
+        !encode_map(kMapQkv, &maps.v, v, 128))
         return ATTN_ERR_CUDA;
     // d <= 64 stages bias tiles through shared memory by TMA; d = 128 reads bias rows directly
-    if (bias != nullptr && d <= 64 && !encode_bias_map(&maps.bias, bias)) return ATTN_ERR_CUDA;
+    if (bias != nullptr && d <= 64 && !encode_map(kMapBias, &maps.bias, bias, 128)) return ATTN_ERR_CUDA;
     unsigned int* status = status_word_ptr();
     if (status == nullptr) return ATTN_ERR_CUDA;
 
@@ -705,7 +761,8 @@ attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, co
     attn_tensor_t pq = view(q, 0, Tq), pk = view(k, 0, Tk), pv = view(v, 0, Tk), po = view(out, 0, Tq);
     Maps maps;
     std::memset(&maps, 0, sizeof(maps));
-    if (!encode_qkv_map(&maps.q, &pq) || !encode_qkv_map(&maps.k, &pk) || !encode_qkv_map(&maps.v, &pv))
+    if (!encode_map(kMapQkv, &maps.q, &pq, 128) || !encode_map(kMapQkv, &maps.k, &pk, 128) ||
+        !encode_map(kMapQkv, &maps.v, &pv, 128))
         return ATTN_ERR_CUDA;
     unsigned int* status = status_word_ptr();
     if (status == nullptr) return ATTN_ERR_CUDA;
@@ -826,9 +883,10 @@ attn_status_t attn_bwd_ex(const attn_tensor_t* q, const attn_tensor_t* k, const 
     tp.window_left = (mods_on && mods->window_left >= 0) ? mods->window_left : -1;
     if (tp.status == nullptr) return ATTN_ERR_CUDA;
     BwdMaps m;
-    if (!encode_qkv_map(&m.q64, q, 64) || !encode_qkv_map(&m.k128, k, 128) || !encode_qkv_map(&m.v128, v, 128) ||
-        !encode_qkv_map(&m.do64, dout, 64) || !encode_qkv_map(&m.q128, q, 128) || !encode_qkv_map(&m.k64, k, 64) ||
-        !encode_qkv_map(&m.v64, v, 64) || !encode_qkv_map(&m.do128, dout, 128))
+    if (!encode_map(kMapQkv, &m.q64, q, 64) || !encode_map(kMapQkv, &m.k128, k, 128) ||
+        !encode_map(kMapQkv, &m.v128, v, 128) || !encode_map(kMapQkv, &m.do64, dout, 64) ||
+        !encode_map(kMapQkv, &m.q128, q, 128) || !encode_map(kMapQkv, &m.k64, k, 64) ||
+        !encode_map(kMapQkv, &m.v64, v, 64) || !encode_map(kMapQkv, &m.do128, dout, 128))
         return ATTN_ERR_CUDA;
     cudaError_t e = q->dtype == ATTN_BF16
                         ? launch_bwd_tc_dtype<__nv_bfloat16>(static_cast<int>(d), causal != 0, mods_on, m, tp, stream)
@@ -927,7 +985,8 @@ attn_status_t attn_fwd_fp8(const attn_tensor_t* q, const attn_tensor_t* k, const
 
     Maps maps;
     std::memset(&maps, 0, sizeof(maps));
-    if (!encode_e4m3_map(&maps.q, q) || !encode_e4m3_map(&maps.k, k) || !encode_e4m3_vt_map(&maps.v, v_t))
+    if (!encode_map(kMapE4m3, &maps.q, q, 128) || !encode_map(kMapE4m3, &maps.k, k, 128) ||
+        !encode_map(kMapE4m3Vt, &maps.v, v_t, 128))
         return ATTN_ERR_CUDA;
     unsigned int* status = status_word_ptr();
     if (status == nullptr) return ATTN_ERR_CUDA;

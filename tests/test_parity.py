@@ -136,6 +136,24 @@ def test_strided_views():
     assert_close_to_oracle(out_buf.transpose(1, 2), lse, o_ref, l_ref, torch.bfloat16, "strided")
 
 
+def test_same_storage_in_two_layouts():
+    """One storage read back to back as [B, H, N, d] and as a transposed [B, N, H, d] view: the
+    same base pointer and shape with other strides must not reuse the first call's tensor maps."""
+    B, H, N, d = 2, 4, 256, 64
+    g = torch.Generator().manual_seed(11)
+    dev = torch.device("cuda")
+    bufs = [torch.randn(B * H * N * d, generator=g).to(torch.float16).to(dev) for _ in range(3)]
+    for layout in ("bhnd", "bnhd", "bhnd"):
+        if layout == "bhnd":
+            q, k, v = (x.view(B, H, N, d) for x in bufs)
+        else:
+            q, k, v = (x.view(B, N, H, d).transpose(1, 2) for x in bufs)
+        o, lse = attn_fwd(q, k, v, causal=True)
+        torch.cuda.synchronize()
+        o_ref, l_ref = sdpa_forward(q.cpu(), k.cpu(), v.cpu(), causal=True)
+        assert_close_to_oracle(o, lse, o_ref, l_ref, torch.float16, f"layout {layout}")
+
+
 def test_evoformer_column_gated_attention():
     """Column-wise gated self-attention of an Evoformer MSA block (the gated Evoformer variant of
     the FLASHLIGHT summary, along the other axis): the MSA activations are [R, C, H, d] and each
