@@ -33,9 +33,11 @@
 //   WG1 (warps 4-7)   the same for Q1.
 //   WG2 (warps 8-11)  epilogue: O/l, gate, rounding, stores of O and lse; at
 //                     d = 128 also the correction (the O rescale above).
-//   warp 12           tcgen05.mma issuer (one thread); allocates tensor memory.
+//   warp 12           tcgen05.mma issuer (one elected lane); allocates tensor memory.
+//                     Without causal masking at d <= 64 it issues only Q0's MMAs and
+//                     warp 14 those of Q1 (one issuer per query tile).
 //   warp 13           TMA producer: Q0, Q1 per unit, K and V tiles into rings.
-//   warps 14-15       idle (they complete warpgroup 3's register hand-back).
+//   warps 14-15       otherwise idle (they complete warpgroup 3's register hand-back).
 //
 // Tensor memory (128 lanes = query rows, 512 columns):
 //   d <= 64:  S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O0 [384,384+d) O1 [384+d, 384+2d)
@@ -377,6 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     using C = Cfg<D, FP8>;
     static_assert(!FP8 || (!HAS_BIAS && !HAS_GATE && !MODS), "e4m3 inputs: plain path only");
     constexpr int ST = C::kStages;
+    // Non-causal with P in its own columns (d <= 64): one MMA issuer per query tile (warps 12 and
+    // 14), each releasing every K / V stage and the drain once.  Both tiles take the same key
+    // tiles there.  (Causal units, where tile 1 takes one more key tile, keep one issuer: the
+    // per-tile form measured slower on them.)
+    constexpr bool kTileIssuers = C::kSeparateP && !CAUSAL;
+    constexpr uint32_t kReleases = kTileIssuers ? 2 : 1;
     // operand format bits of the instruction descriptor: 1 selects bf16 (kind::f16); e4m3 is 0
     constexpr bool kBF16 = !FP8 && std::is_same<T, __nv_bfloat16>::value;
 
@@ -408,11 +416,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < ST; ++s) {
             mbar_init(&sh.k_full[s], 1);
-            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.k_empty[s], kReleases);
             mbar_init(&sh.v_full[s], 1);
-            mbar_init(&sh.v_empty[s], 1);
+            mbar_init(&sh.v_empty[s], kReleases);
         }
-        mbar_init(&sh.drain, 1);
+        mbar_init(&sh.drain, kReleases);
         mbar_init(&sh.never, 1);
         for (int i = 0; i < 2; ++i)
             for (int b = 0; b < 2; ++b) {
@@ -538,17 +546,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (bc[i] > s)
                             drain_phase(&sh.bias_full[i][s], ((bc[i] - 1 - s) / BC::kStages) & 1, p.status);
             }
-        } else if (warp == 12) {
-            // ============================================================ MMA issuer
+        } else if (warp == 12 || (kTileIssuers && warp == 14)) {
+            // ============================================================ MMA issuer(s)
             constexpr uint32_t idesc_s = instr_desc_f16(kBF16, kBlockM, kBlockN, false);
             // (e4m3: V^T is K-major, like K in S; 16-bit V is N-major)
             constexpr uint32_t idesc_o = instr_desc_f16(kBF16, kBlockM, D, !FP8);
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t k_addr = smem_u32(sK);
             const uint32_t v_addr = smem_u32(sV);
-            constexpr uint32_t kColS[2] = {C::kColS0, C::kColS1};
-            constexpr uint32_t kColP[2] = {C::kColP0, C::kColP1};
-            constexpr uint32_t kColO[2] = {C::kColO0, C::kColO1};
+            // (columns by select, not by indexing a local array with a runtime tile index)
+            auto col_s = [](int i) { return i ? C::kColS1 : C::kColS0; };
+            auto col_p = [](int i) { return i ? C::kColP1 : C::kColP0; };
+            auto col_o = [](int i) { return i ? C::kColO1 : C::kColO0; };
             // Descriptors are affine in the start address (bits [0,14) hold address / 16 and
             // shared addresses stay below 256 KB), so each step adds a constant to a base.
             const uint64_t dq = smem_desc(q_addr, 16, C::kSBO, C::kLayout);
@@ -576,9 +585,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < D / C::kK; ++kk) {
                         const uint32_t off = C::kstep(kk);
                         if constexpr (FP8)
-                            mma_ss_f8(tmem + kColS[i], desc(qb + off, dq_hi), desc(kb + off, dk_hi), idesc_s, kk > 0 ? 1u : 0u);
+                            mma_ss_f8(tmem + col_s(i), desc(qb + off, dq_hi), desc(kb + off, dk_hi), idesc_s, kk > 0 ? 1u : 0u);
                         else
-                            mma_ss(tmem + kColS[i], desc(qb + off, dq_hi), desc(kb + off, dk_hi), idesc_s, kk > 0 ? 1u : 0u);
+                            mma_ss(tmem + col_s(i), desc(qb + off, dq_hi), desc(kb + off, dk_hi), idesc_s, kk > 0 ? 1u : 0u);
                     }
                 }
             };
@@ -591,9 +600,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < kBlockN / C::kK; ++kk) {
                         const uint64_t vk = desc(vb + (FP8 ? ((kk * 32) >> 4) : ((kk * C::kK * C::kRowBytes) >> 4)), dv_hi);
                         if constexpr (FP8)
-                            mma_ts_f8(tmem + kColO[i], tmem + kColP[i] + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
+                            mma_ts_f8(tmem + col_o(i), tmem + col_p(i) + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
                         else
-                            mma_ts(tmem + kColO[i], tmem + kColP[i] + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
+                            mma_ts(tmem + col_o(i), tmem + col_p(i) + kk * 8, vk, idesc_o, (acc || kk > 0) ? 1u : 0u);
                     }
                 }
             };
@@ -615,54 +624,131 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 issue_s(i, kpos % ST);
                 commit(&sh.s_full[i]);
-                if (i == 1) commit(&sh.k_empty[kpos % ST]);
+                if (kTileIssuers || i == 1) commit(&sh.k_empty[kpos % ST]);
                 if (nkv_i == 1) commit(&sh.q_empty[i]);
                 return true;
             };
-            // d <= 64 issues S_i(0) of the next unit right after this unit's last PV_i rather than
-            // after both tiles' last PVs, so tile 0's softmax restarts one PV group earlier.
-            // Issued after that PV, S_i(0) needs no further ordering: its commit covers the PV.
-            bool early[2] = {false, false};
-            for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
-                const Unit U = decode_unit<CAUSAL, MODS>(u, p);
-                const int u_next = unit_at(uit + 1);
-                int nkv_next[2] = {0, 0};      // 0: no next unit
-                if (C::kSeparateP && u_next < p.num_units) {
-                    const Unit Un = decode_unit<CAUSAL, MODS>(u_next, p);
-                    nkv_next[0] = Un.nkv0;
-                    nkv_next[1] = Un.nkv1;
-                }
-                // S0(0), S1(0), unless issued at the end of the previous unit
-                if (!early[0] && !issue_first_s(0, U.nkv0, kc, uit & 1)) break;
-                if (!early[1] && !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
-                early[0] = early[1] = false;
-                for (int j = 0; j < U.nkv1; ++j) {
-                    const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
-                    const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
-                    if constexpr (C::kSeparateP) {
-                        // S0(j+1), S1(j+1) as soon as the softmax has read S(j); then PV0(j), PV1(j)
-                        if (j + 1 < U.nkv0) {
-                            if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
-                            ++sf_cnt[0];
+            if constexpr (kTileIssuers) {
+                // One query tile per issuing warp: S_ti(j+1) as soon as the softmax has read
+                // S_ti(j), then PV_ti(j); the next unit's S_ti(0) right behind the unit's last PV_ti.
+                const int ti = warp == 12 ? 0 : 1;
+                uint32_t pv_n = 0, sf_n = 0;
+                bool early_t = false;
+                for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
+                    const Unit U = decode_unit<CAUSAL, MODS>(u, p);
+                    const int nkv = U.nkv1;          // == nkv0 without causal masking
+                    const int u_next = unit_at(uit + 1);
+                    const int nkv_next = u_next < p.num_units ? decode_unit<CAUSAL, MODS>(u_next, p).nkv1 : 0;
+                    if (!early_t && !issue_first_s(ti, nkv, kc, uit & 1)) break;
+                    early_t = false;
+                    for (int j = 0; j < nkv; ++j) {
+                        const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
+                        const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
+                        if (j + 1 < nkv) {
+                            if (!W(&sh.s_free[ti], sf_n & 1)) break;
+                            ++sf_n;
                             if (!W(&sh.k_full[kst], kph)) break;
                             tc_fence_after();
-                            issue_s(0, kst);
-                            commit(&sh.s_full[0]);
-                            if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
-                        }
-                        if (j + 1 < U.nkv1) {
-                            if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
-                            ++sf_cnt[1];
-                            // (K(j+1) has been waited for by S0(j+1) unless tile 0 ends at j: only
-                            // causal units give tile 1 one more key tile)
-                            if (j + 1 >= U.nkv0 && !W(&sh.k_full[kst], kph)) break;
-                            tc_fence_after();
-                            issue_s(1, kst);
-                            commit(&sh.s_full[1]);
+                            issue_s(ti, kst);
+                            commit(&sh.s_full[ti]);
                             commit(&sh.k_empty[kst]);
-                            if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
+                            if (j + 2 == nkv) commit(&sh.q_empty[ti]);
                         }
-                        if (j < U.nkv0) {
+                        if (!W(&sh.pv_ready[ti], pv_n & 1)) break;
+                        ++pv_n;
+                        if (j == 0 && uit > 0 && !W(&sh.o_free[ti], (uit - 1) & 1)) break;
+                        if (!W(&sh.v_full[vst], vph)) break;
+                        tc_fence_after();
+                        issue_pv(ti, vst, j > 0);
+                        commit(&sh.o_done[ti]);
+                        commit(&sh.v_empty[vst]);
+                        if (j + 1 == nkv) {
+                            commit(&sh.o_final[ti]);
+                            if (nkv_next > 0) {
+                                if (!issue_first_s(ti, nkv_next, kc + nkv, (uit + 1) & 1)) break;
+                                early_t = true;
+                            }
+                        }
+                    }
+                    kc += nkv;
+                    vc += nkv;
+                }
+            } else {
+                // d <= 64 issues S_i(0) of the next unit right after this unit's last PV_i rather than
+                // after both tiles' last PVs, so tile 0's softmax restarts one PV group earlier.
+                // Issued after that PV, S_i(0) needs no further ordering: its commit covers the PV.
+                bool early[2] = {false, false};
+                for (int u = unit_at(0); ok && u < p.num_units; u = unit_at(++uit)) {
+                    const Unit U = decode_unit<CAUSAL, MODS>(u, p);
+                    const int u_next = unit_at(uit + 1);
+                    int nkv_next[2] = {0, 0};      // 0: no next unit
+                    if (C::kSeparateP && u_next < p.num_units) {
+                        const Unit Un = decode_unit<CAUSAL, MODS>(u_next, p);
+                        nkv_next[0] = Un.nkv0;
+                        nkv_next[1] = Un.nkv1;
+                    }
+                    // S0(0), S1(0), unless issued at the end of the previous unit
+                    if (!early[0] && !issue_first_s(0, U.nkv0, kc, uit & 1)) break;
+                    if (!early[1] && !issue_first_s(1, U.nkv1, kc, uit & 1)) break;
+                    early[0] = early[1] = false;
+                    for (int j = 0; j < U.nkv1; ++j) {
+                        const uint32_t vst = (vc + j) % ST, vph = ((vc + j) / ST) & 1;
+                        const uint32_t kn = kc + j + 1, kst = kn % ST, kph = (kn / ST) & 1;
+                        if constexpr (C::kSeparateP) {
+                            // S0(j+1), S1(j+1) as soon as the softmax has read S(j); then PV0(j), PV1(j)
+                            if (j + 1 < U.nkv0) {
+                                if (!W(&sh.s_free[0], sf_cnt[0] & 1)) break;
+                                ++sf_cnt[0];
+                                if (!W(&sh.k_full[kst], kph)) break;
+                                tc_fence_after();
+                                issue_s(0, kst);
+                                commit(&sh.s_full[0]);
+                                if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
+                            }
+                            if (j + 1 < U.nkv1) {
+                                if (!W(&sh.s_free[1], sf_cnt[1] & 1)) break;
+                                ++sf_cnt[1];
+                                // (K(j+1) has been waited for by S0(j+1) unless tile 0 ends at j: only
+                                // causal units give tile 1 one more key tile)
+                                if (j + 1 >= U.nkv0 && !W(&sh.k_full[kst], kph)) break;
+                                tc_fence_after();
+                                issue_s(1, kst);
+                                commit(&sh.s_full[1]);
+                                commit(&sh.k_empty[kst]);
+                                if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
+                            }
+                            if (j < U.nkv0) {
+                                if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
+                                ++pv_cnt[0];
+                                if (j == 0 && uit > 0 && !W(&sh.o_free[0], (uit - 1) & 1)) break;
+                                if (!W(&sh.v_full[vst], vph)) break;
+                                tc_fence_after();
+                                issue_pv(0, vst, j > 0);
+                                commit(&sh.o_done[0]);
+                                if (j + 1 == U.nkv0) commit(&sh.o_final[0]);
+                                if (j + 1 == U.nkv0 && nkv_next[0] > 0) {
+                                    if (!issue_first_s(0, nkv_next[0], kc + U.nkv1, (uit + 1) & 1))
+                                        break;
+                                    early[0] = true;
+                                }
+                            }
+                            if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
+                            ++pv_cnt[1];
+                            if (j == 0 && uit > 0 && !W(&sh.o_free[1], (uit - 1) & 1)) break;
+                            if (j >= U.nkv0 && !W(&sh.v_full[vst], vph)) break;   // else seen by PV0(j)
+                            tc_fence_after();
+                            issue_pv(1, vst, j > 0);
+                            commit(&sh.o_done[1]);
+                            commit(&sh.v_empty[vst]);
+                            if (j + 1 == U.nkv1) commit(&sh.o_final[1]);
+                            if (j + 1 == U.nkv1 && nkv_next[1] > 0) {
+                                if (!issue_first_s(1, nkv_next[1], kc + U.nkv1, (uit + 1) & 1))
+                                    break;
+                                early[1] = true;
+                            }
+                            continue;
+                        }
+                        if (j < U.nkv0) {   // PV0(j)
                             if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
                             ++pv_cnt[0];
                             if (j == 0 && uit > 0 && !W(&sh.o_free[0], (uit - 1) & 1)) break;
@@ -670,65 +756,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                             issue_pv(0, vst, j > 0);
                             commit(&sh.o_done[0]);
-                            if (j + 1 == U.nkv0) commit(&sh.o_final[0]);
-                            if (j + 1 == U.nkv0 && nkv_next[0] > 0) {
-                                if (!issue_first_s(0, nkv_next[0], kc + U.nkv1, (uit + 1) & 1))
-                                    break;
-                                early[0] = true;
-                            }
                         }
+                        if (j + 1 < U.nkv0) {   // S0(j+1)
+                            if (!W(&sh.k_full[kst], kph)) break;
+                            tc_fence_after();
+                            issue_s(0, kst);
+                            commit(&sh.s_full[0]);
+                            if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
+                        }
+                        // PV1(j)
                         if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
                         ++pv_cnt[1];
                         if (j == 0 && uit > 0 && !W(&sh.o_free[1], (uit - 1) & 1)) break;
-                        if (j >= U.nkv0 && !W(&sh.v_full[vst], vph)) break;   // else seen by PV0(j)
+                        if (!W(&sh.v_full[vst], vph)) break;
                         tc_fence_after();
                         issue_pv(1, vst, j > 0);
                         commit(&sh.o_done[1]);
                         commit(&sh.v_empty[vst]);
-                        if (j + 1 == U.nkv1) commit(&sh.o_final[1]);
-                        if (j + 1 == U.nkv1 && nkv_next[1] > 0) {
-                            if (!issue_first_s(1, nkv_next[1], kc + U.nkv1, (uit + 1) & 1))
-                                break;
-                            early[1] = true;
+                        if (j + 1 < U.nkv1) {   // S1(j+1)
+                            if (!W(&sh.k_full[kst], kph)) break;
+                            tc_fence_after();
+                            issue_s(1, kst);
+                            commit(&sh.s_full[1]);
+                            commit(&sh.k_empty[kst]);
+                            if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
                         }
-                        continue;
                     }
-                    if (j < U.nkv0) {   // PV0(j)
-                        if (!W(&sh.pv_ready[0], pv_cnt[0] & 1)) break;
-                        ++pv_cnt[0];
-                        if (j == 0 && uit > 0 && !W(&sh.o_free[0], (uit - 1) & 1)) break;
-                        if (!W(&sh.v_full[vst], vph)) break;
-                        tc_fence_after();
-                        issue_pv(0, vst, j > 0);
-                        commit(&sh.o_done[0]);
-                    }
-                    if (j + 1 < U.nkv0) {   // S0(j+1)
-                        if (!W(&sh.k_full[kst], kph)) break;
-                        tc_fence_after();
-                        issue_s(0, kst);
-                        commit(&sh.s_full[0]);
-                        if (j + 2 == U.nkv0) commit(&sh.q_empty[0]);
-                    }
-                    // PV1(j)
-                    if (!W(&sh.pv_ready[1], pv_cnt[1] & 1)) break;
-                    ++pv_cnt[1];
-                    if (j == 0 && uit > 0 && !W(&sh.o_free[1], (uit - 1) & 1)) break;
-                    if (!W(&sh.v_full[vst], vph)) break;
-                    tc_fence_after();
-                    issue_pv(1, vst, j > 0);
-                    commit(&sh.o_done[1]);
-                    commit(&sh.v_empty[vst]);
-                    if (j + 1 < U.nkv1) {   // S1(j+1)
-                        if (!W(&sh.k_full[kst], kph)) break;
-                        tc_fence_after();
-                        issue_s(1, kst);
-                        commit(&sh.s_full[1]);
-                        commit(&sh.k_empty[kst]);
-                        if (j + 2 == U.nkv1) commit(&sh.q_empty[1]);
-                    }
+                    kc += U.nkv1;
+                    vc += U.nkv1;
                 }
-                kc += U.nkv1;
-                vc += U.nkv1;
             }
             // drain: all MMAs complete before tensor memory is released
             commit(&sh.drain);

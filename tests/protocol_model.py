@@ -1,7 +1,8 @@
 """A model of the forward kernel's mbarrier protocol, checked under random interleavings.
 
 The kernel in exact_attention_sdpa_b200/csrc/attn_fwd_kernel.cuh moves every tile between its
-roles (TMA producer, MMA issuer, two softmax warpgroups, epilogue warpgroup) through
+roles (TMA producer, MMA issuer -- one per query tile for non-causal d <= 64 --, two softmax
+warpgroups, epilogue warpgroup) through
 mbarriers whose waits name a phase only by its parity.  compute-sanitizer cannot run on the
 machines these kernels are measured on, so this module re-states the protocol as it is written
 in the kernel, one actor per warp, and executes it on the CPU under random schedules:
@@ -116,6 +117,11 @@ def random_units(rng: random.Random, causal: bool, n_units: int, max_tiles: int 
     return out
 
 
+def tile_issuers(cfg: "Config") -> bool:
+    """The kernel's kTileIssuers: separate P columns (d <= 64) without causal masking."""
+    return cfg.separate_p and not cfg.causal
+
+
 # ---------------------------------------------------------------------------------------- state
 class State:
     def __init__(self, cfg: Config):
@@ -125,9 +131,12 @@ class State:
         self.q_full = [B(f"q_full{i}", 1) for i in range(2)]
         self.q_empty = [B(f"q_empty{i}", 1) for i in range(2)]
         self.k_full = [B(f"k_full{s}", 1) for s in range(ST)]
-        self.k_empty = [B(f"k_empty{s}", 1) for s in range(ST)]
+        # non-causal d <= 64: one issuer per query tile, each releasing every K / V stage and the
+        # drain once
+        rel = 2 if tile_issuers(cfg) else 1
+        self.k_empty = [B(f"k_empty{s}", rel) for s in range(ST)]
         self.v_full = [B(f"v_full{s}", 1) for s in range(ST)]
-        self.v_empty = [B(f"v_empty{s}", 1) for s in range(ST)]
+        self.v_empty = [B(f"v_empty{s}", rel) for s in range(ST)]
         self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
         self.s_free = [B(f"s_free{i}", 128) for i in range(2)]
         # separate P (d <= 64): the softmax rescales O itself and alone releases PV_i(j); P inside S
@@ -140,8 +149,9 @@ class State:
         self.stats_full = [B(f"stats_full{i}", 128) for i in range(2)]
         self.bias_full = [[B(f"bias_full{i}.{s}", 1) for s in range(BS)] for i in range(2)]
         self.bias_empty = [[B(f"bias_empty{i}.{s}", 128) for s in range(BS)] for i in range(2)]
-        self.drain = B("drain", 1)
-        self.teardown = B("teardown", 14)             # __syncthreads before tensor memory is freed
+        self.drain = B("drain", rel)
+        # __syncthreads before tensor memory is freed (one arrival per modelled warp)
+        self.teardown = B("teardown", 15 if tile_issuers(cfg) else 14)
         self.abort = False                            # the CTA's abort flag
         # buffers (version tags)
         self.sQ = [None, None]
@@ -268,16 +278,16 @@ def producer(st: State):
     yield from teardown(st)
 
 
-def s_mma(st: State, i: int, k: int, j: int, kst: int, key_tile: int):
+def s_mma(st: State, i: int, k: int, j: int, kst: int, key_tile: int, thread: str = "mma"):
     def run(s):
         s.expect(f"S{i}({k},{j}) reads Q{i}", s.sQ[i], k)
         s.expect(f"S{i}({k},{j}) reads K stage {kst}", s.sK[kst], key_tile)
         for q in range(4):
             s.tS[i][q] = ("S", k, j)
-    return Issue("mma", f"S{i}({k},{j})", run)
+    return Issue(thread, f"S{i}({k},{j})", run)
 
 
-def pv_mma(st: State, i: int, k: int, j: int, vst: int, key_tile: int):
+def pv_mma(st: State, i: int, k: int, j: int, vst: int, key_tile: int, thread: str = "mma"):
     def run(s):
         s.expect(f"PV{i}({k},{j}) reads V stage {vst}", s.sV[vst], key_tile)
         for q in range(4):
@@ -292,7 +302,85 @@ def pv_mma(st: State, i: int, k: int, j: int, vst: int, key_tile: int):
                 if o["rescaled"] != j:
                     raise ProtocolError(f"PV{i}({k},{j}) runs before O{i} was rescaled for alpha({j})")
             s.tO[i][q] = {"unit": k, "done": j, "rescaled": o["rescaled"] if j else 0, "read": False}
-    return Issue("mma", f"PV{i}({k},{j})", run)
+    return Issue(thread, f"PV{i}({k},{j})", run)
+
+
+def mma_tile_issuer(st: State, ti: int):
+    """Non-causal d <= 64: the issuing warp of query tile ti (warp 12 for tile 0, warp 14 for
+    tile 1).  S_ti(j+1) as soon as S_ti(j) was read, then PV_ti(j); the next unit's S_ti(0) right
+    behind the unit's last PV_ti; one release of every K and V stage it read, one commit to the
+    drain.  Both tiles take the same key tiles (no causal masking)."""
+    cfg, ST = st.cfg, st.cfg.stages
+    thread = f"mma{ti}"
+    kc = vc = 0
+    pv_n = sf_n = 0
+    early = False
+    n_units = len(cfg.units)
+    ok = True
+
+    def W(bar, parity, phase):
+        nonlocal ok
+        if ok:
+            ok = yield Wait(bar, parity, phase)
+        return ok
+
+    def first_s(k, kpos, nkv):
+        if not (yield from W(st.q_full[ti], k & 1, k)):
+            return False
+        if not (yield from W(st.k_full[kpos % ST], (kpos // ST) & 1, kpos // ST)):
+            return False
+        yield s_mma(st, ti, k, 0, kpos % ST, kpos, thread)
+        yield Commit(thread, st.s_full[ti])
+        yield Commit(thread, st.k_empty[kpos % ST])
+        if nkv == 1:
+            yield Commit(thread, st.q_empty[ti])
+        return True
+
+    for k in range(n_units):
+        nkv = cfg.units[k][ti]
+        nkv_next = cfg.units[k + 1][ti] if k + 1 < n_units else 0
+        if not ok:
+            break
+        if not early and not (yield from first_s(k, kc, nkv)):
+            break
+        early = False
+        for j in range(nkv):
+            vn, kn = vc + j, kc + j + 1
+            vst, vph, kst, kph = vn % ST, (vn // ST) & 1, kn % ST, (kn // ST) & 1
+            if j + 1 < nkv:
+                if not (cfg.plant == "no_s_free_wait" and ti == 0) and \
+                        not (yield from W(st.s_free[ti], sf_n & 1, sf_n)):
+                    break
+                sf_n += 1
+                if cfg.plant != "s_skips_k_wait" and not (yield from W(st.k_full[kst], kph, kn // ST)):
+                    break
+                yield s_mma(st, ti, k, j + 1, kst, kn, thread)
+                yield Commit(thread, st.s_full[ti])
+                yield Commit(thread, st.k_empty[kst])
+                if j + 2 == nkv:
+                    yield Commit(thread, st.q_empty[ti])
+            if not (yield from W(st.pv_ready[ti], pv_n & 1, pv_n)):
+                break
+            pv_n += 1
+            if j == 0 and k > 0 and not (yield from W(st.o_free[ti], (k - 1) & 1, k - 1)):
+                break
+            if not (yield from W(st.v_full[vst], vph, vn // ST)):
+                break
+            yield pv_mma(st, ti, k, j, vst, vn, thread)
+            yield Commit(thread, st.o_done[ti])
+            yield Commit(thread, st.v_empty[vst])
+            if j + 1 == nkv:
+                yield Commit(thread, st.o_final[ti])
+                if nkv_next > 0:
+                    if not (yield from first_s(k + 1, kc + nkv, nkv_next)):
+                        break
+                    early = True
+        kc += nkv
+        vc += nkv
+    if cfg.plant != "no_mma_drain":
+        yield Commit(thread, st.drain)
+        yield Wait(st.drain, 0, 0, drain=True)
+    yield from teardown(st)
 
 
 def mma_issuer(st: State):
@@ -597,7 +685,12 @@ def epilogue_warp(st: State, q: int):
 
 
 def kernel_roles(st: State) -> dict:
-    roles = {"tma": producer(st), "mma": mma_issuer(st)}
+    roles = {"tma": producer(st)}
+    if tile_issuers(st.cfg):
+        roles["mma0"] = mma_tile_issuer(st, 0)
+        roles["mma1"] = mma_tile_issuer(st, 1)
+    else:
+        roles["mma"] = mma_issuer(st)
     for i in range(2):
         for q in range(4):
             roles[f"softmax{i}.{q}"] = softmax_warp(st, i, q)

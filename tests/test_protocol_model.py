@@ -55,7 +55,8 @@ def test_single_tile_units_back_to_back():
         pm.run(cfg, seed=rep)
 
 
-ROLES = ["tma", "mma"] + [f"softmax{i}.{q}" for i in range(2) for q in range(4)] + [f"epi.{q}" for q in range(4)]
+ROLES = ["tma", "mma", "mma0", "mma1"] + [f"softmax{i}.{q}" for i in range(2) for q in range(4)] + \
+    [f"epi.{q}" for q in range(4)]
 
 
 @pytest.mark.parametrize("sep,causal,stages,bias", [(True, True, 3, 0), (True, False, 4, 2), (True, True, 3, 1),
@@ -80,8 +81,9 @@ def test_a_timeout_at_any_wait_drains_and_exits(sep, causal, stages, bias):
 def test_model_finds_a_missing_drain(plant):
     for rep in range(200):
         rng = random.Random(rep)
-        cfg = pm.Config(separate_p=rep % 2 == 0, causal=True, stages=3 if rep % 2 == 0 else 2,
-                        units=pm.random_units(rng, True, 2, max_tiles=3), plant=plant,
+        causal = rep % 4 != 0         # every other d <= 64 run non-causal: the two tile issuers
+        cfg = pm.Config(separate_p=rep % 2 == 0, causal=causal, stages=3 if rep % 2 == 0 else 2,
+                        units=pm.random_units(rng, causal, 2, max_tiles=3), plant=plant,
                         timeout=(rng.choice(ROLES), rng.randint(0, 4)))
         try:
             pm.run(cfg, seed=rep)
@@ -95,6 +97,7 @@ PLANTS = {
     "empty_parity": True,           # producer waits the K/V release of the wrong phase
     "no_s_free_wait": True,         # S_0(j+1) issued before the softmax read S_0(j)
     "s1_skips_k_wait": True,        # S_1(j+1) for the extra key tile of a causal unit without K's wait
+    "s_skips_k_wait": True,         # a tile issuer (non-causal d <= 64) issues S_i(j+1) without K's wait
     "s_before_pv": False,           # d = 128: S_0(j+1) overwrites P_0(j) before PV_0(j)
     "rescale_before_o_done": True,  # O_i rescaled before PV_i(j-1) completed
     "no_o_done_wait": True,         # P_i(j) written while PV_i(j-1) may still read P_i(j-1)
@@ -120,10 +123,11 @@ def test_model_finds_planted_mistakes(plant):
 
 
 def test_softmax_o_free_wait_is_a_second_guard():
-    """The softmax's wait for the previous epilogue (o_free) before it publishes a unit's final
-    m, l is implied by the rest of the protocol: the next unit's first S_i is issued only after
-    PV_i(0) of the current unit, which waited for the epilogue two units back.  Without the wait
-    the model still finds no stale read; the kernel keeps it as a cheap second guard."""
+    """One MMA issuer for both tiles (causal d <= 64, and d = 128): the softmax's wait for the
+    previous epilogue (o_free) before it publishes a unit's final m, l is implied by the rest of
+    the protocol -- the next unit's first S_i is issued only after PV_i(0) of the current unit,
+    which waited for the epilogue two units back.  Without the wait the model finds no stale
+    read; the kernel keeps it as a second guard."""
     for rep in range(200):
         rng = random.Random(rep)
         sep = rep % 2 == 0
@@ -133,6 +137,22 @@ def test_softmax_o_free_wait_is_a_second_guard():
         pm.run(cfg, seed=rep)
 
 
+def test_softmax_o_free_wait_is_needed_with_tile_issuers():
+    """One MMA issuer per tile (non-causal d <= 64): a tile's issuer does not wait for the other
+    tile's PVs, so a softmax warpgroup can run two units ahead of the epilogue, and without the
+    o_free wait its statistics overtake the epilogue's reads; the model must find that."""
+    for rep in range(400):
+        rng = random.Random(rep)
+        cfg = pm.Config(separate_p=True, causal=False, stages=3,
+                        units=pm.random_units(rng, False, rng.randint(2, 6), max_tiles=2),
+                        plant="stats_no_o_free_wait")
+        try:
+            pm.run(cfg, seed=rep)
+        except pm.ProtocolError:
+            return
+    pytest.fail("the missing o_free wait went unnoticed in 400 schedules")
+
+
 def test_model_barriers_match_the_kernel_source():
     # The model must know every mbarrier the kernel initialises, with the same arrival count;
     # a barrier added to or re-counted in the kernel without the model fails here.
@@ -140,13 +160,17 @@ def test_model_barriers_match_the_kernel_source():
     import re
     src = open(os.path.join(os.path.dirname(__file__), "..", "exact_attention_sdpa_b200", "csrc",
                             "attn_fwd_kernel.cuh")).read()
-    for sep in (True, False):
+    assert "constexpr bool kTileIssuers = C::kSeparateP && !CAUSAL;" in src
+    assert "constexpr uint32_t kReleases = kTileIssuers ? 2 : 1;" in src
+    for sep, causal in ((True, True), (True, False), (False, True)):
         found = {}
         for name, expr in re.findall(r"mbar_init\(&sh\.(\w+)(?:\[[^\]]*\])*,\s*([^;]+)\);", src):
-            # C::kPvArrivals: the softmax's 128 arrivals, plus the correction's 128 at d = 128
-            found[name] = eval(expr.strip().replace("C::kPvArrivals", "kPv"), {"kBlockM": 128, "kPv": 128 if sep else 256})
+            # C::kPvArrivals: the softmax's 128 arrivals, plus the correction's 128 at d = 128;
+            # kReleases: one K/V/drain release per MMA issuer
+            found[name] = eval(expr.strip().replace("C::kPvArrivals", "kPv"),
+                               {"kBlockM": 128, "kPv": 128 if sep else 256, "kReleases": 2 if sep and not causal else 1})
         found.pop("never")            # stall-injection target: nothing ever arrives on it
-        check_barriers(found, pm.State(pm.Config(units=[(1, 1)], bias_stages=1, separate_p=sep)))
+        check_barriers(found, pm.State(pm.Config(units=[(1, 1)], bias_stages=1, separate_p=sep, causal=causal)))
 
 
 def check_barriers(found, st):
