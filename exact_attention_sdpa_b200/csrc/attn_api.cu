@@ -779,16 +779,32 @@ attn_status_t attn_fwd_varlen(const attn_tensor_t* q, const attn_tensor_t* k, co
         p.n_kv_tiles = 1;
         p.head_group = static_cast<int>(H);
         p.n_seq = static_cast<int>(c1 - c0);
-        int64_t units = 0;
+        // causal with N_q = N_k everywhere: units ordered by query pair across the sequences (the
+        // chunk is sorted by causal work, which for N_q = N_k orders the pair counts, most first)
+        bool level = causal != 0;
+        for (size_t i = c0; i < c1; ++i)
+            level = level && (cu_seqlens_q[order[i] + 1] - cu_seqlens_q[order[i]] ==
+                              cu_seqlens_k[order[i] + 1] - cu_seqlens_k[order[i]]);
+        p.level_order = level ? 1 : 0;
+        auto pairs = [&](int s) { return (p.seq_nq[s] + attn::kRowsPerUnit - 1) / attn::kRowsPerUnit; };
         for (size_t i = c0; i < c1; ++i) {
             const int32_t b = order[i];
             const int s = static_cast<int>(i - c0);
-            p.seq_units[s] = static_cast<int>(units);
             p.seq_q0[s] = cu_seqlens_q[b];
             p.seq_k0[s] = cu_seqlens_k[b];
             p.seq_nq[s] = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
             p.seq_nk[s] = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
-            units += H * ((p.seq_nq[s] + attn::kRowsPerUnit - 1) / attn::kRowsPerUnit);
+        }
+        int64_t units = 0;
+        for (int s = 0; s < p.n_seq; ++s) {
+            p.seq_units[s] = static_cast<int>(units);
+            if (level) {
+                // segment s: the pairs of sequences 0..s beyond those of sequence s + 1
+                const int below = s + 1 < p.n_seq ? pairs(s + 1) : 0;
+                units += static_cast<int64_t>(s + 1) * H * (pairs(s) - below);
+            } else {
+                units += H * pairs(s);
+            }
         }
         if (units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
         p.seq_units[p.n_seq] = static_cast<int>(units);

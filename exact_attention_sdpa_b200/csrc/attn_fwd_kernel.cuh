@@ -98,9 +98,15 @@ struct FwdParams {
     int inject_stall;          // test hook: the MMA warp first waits on a barrier nothing arrives on
     float v_scale;             // e4m3 inputs: the value tensor's scale (the query and key scales are in scale)
     // ragged batch in one launch (n_seq > 0; B = 1 and the tensors are packed [1, H, T, d] views):
-    // sequence s owns query rows seq_q0[s] .. + seq_nq[s] and key rows seq_k0[s] .. + seq_nk[s],
-    // and units seq_units[s] .. seq_units[s + 1] (its query pairs x H, heaviest pairs first)
+    // sequence s owns query rows seq_q0[s] .. + seq_nq[s] and key rows seq_k0[s] .. + seq_nk[s].
+    // level_order == 0: units seq_units[s] .. seq_units[s + 1] are sequence s's query pairs x H,
+    // heaviest pairs first.  level_order == 1 (causal, N_q = N_k in every sequence, sequences
+    // sorted by query pairs, most first): the units of all sequences ordered by query pair,
+    // highest first, which is heaviest first (a causal pair's key tiles depend on its index
+    // only); segment i, units seq_units[i] .. seq_units[i + 1], holds the pairs only sequences
+    // 0..i have, (i + 1) x H units per pair.
     int n_seq;
+    int level_order;
     int seq_units[kMaxSeq + 1];
     int seq_q0[kMaxSeq], seq_k0[kMaxSeq], seq_nq[kMaxSeq], seq_nk[kMaxSeq];
 };
@@ -308,13 +314,23 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
             else hi = mid - 1;
         }
         const int r = u - p.seq_units[lo];
-        U.N = p.seq_nq[lo];
-        U.Nk = p.seq_nk[lo];
-        U.q_base = p.seq_q0[lo];
-        U.k_base = p.seq_k0[lo];
-        const int nqp = (U.N + kRowsPerUnit - 1) / kRowsPerUnit;
-        U.qp = nqp - 1 - r / p.H;
-        U.h = r % p.H;
+        int s = lo;
+        if (p.level_order) {
+            // segment lo: (lo + 1) sequences x H units per query pair, pairs from nqp(lo) - 1 down
+            const int per_pair = (lo + 1) * p.H;
+            const int t = r / per_pair, w = r - t * per_pair;
+            s = w / p.H;
+            U.qp = (p.seq_nq[lo] + kRowsPerUnit - 1) / kRowsPerUnit - 1 - t;
+            U.h = w % p.H;
+        } else {
+            const int nqp = (p.seq_nq[lo] + kRowsPerUnit - 1) / kRowsPerUnit;
+            U.qp = nqp - 1 - r / p.H;
+            U.h = r % p.H;
+        }
+        U.N = p.seq_nq[s];
+        U.Nk = p.seq_nk[s];
+        U.q_base = p.seq_q0[s];
+        U.k_base = p.seq_k0[s];
         U.b = 0;
         U.bh = U.h;
     } else {

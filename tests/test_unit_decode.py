@@ -33,11 +33,19 @@ def decode(u, p):
             else:
                 hi = mid - 1
         r = u - p["seq_units"][lo]
-        U["N"], U["Nk"] = p["seq_nq"][lo], p["seq_nk"][lo]
-        nqp = (U["N"] + ROWS_PER_UNIT - 1) // ROWS_PER_UNIT
-        U["qp"] = nqp - 1 - r // p["H"]
-        U["h"] = r % p["H"]
-        U["seq"] = lo
+        s = lo
+        if p.get("level_order"):
+            per_pair = (lo + 1) * p["H"]
+            t, w = r // per_pair, r % per_pair
+            s = w // p["H"]
+            U["qp"] = (p["seq_nq"][lo] + ROWS_PER_UNIT - 1) // ROWS_PER_UNIT - 1 - t
+            U["h"] = w % p["H"]
+        else:
+            nqp = (p["seq_nq"][lo] + ROWS_PER_UNIT - 1) // ROWS_PER_UNIT
+            U["qp"] = nqp - 1 - r // p["H"]
+            U["h"] = r % p["H"]
+        U["N"], U["Nk"] = p["seq_nq"][s], p["seq_nk"][s]
+        U["seq"] = s
     else:
         BH, G = p["B"] * p["H"], p["head_group"]
         per = G * p["num_q_pairs"]
@@ -125,16 +133,23 @@ def varlen_params(lengths, H, causal):
                       else lengths[b][0] * lengths[b][1])
     order.sort(key=lambda b: -work(b))        # (Python's sort is stable, as std::stable_sort)
     launches = []
+    pairs = lambda b: (lengths[b][0] + ROWS_PER_UNIT - 1) // ROWS_PER_UNIT
     for c0 in range(0, len(order), 64):
         chunk = order[c0:c0 + 64]
+        # causal with N_q = N_k in every sequence: units ordered by query pair across the chunk
+        level = causal and all(lengths[b][0] == lengths[b][1] for b in chunk)
         units, su = 0, []
-        for b in chunk:
+        for i, b in enumerate(chunk):
             su.append(units)
-            units += H * ((lengths[b][0] + ROWS_PER_UNIT - 1) // ROWS_PER_UNIT)
+            if level:
+                below = pairs(chunk[i + 1]) if i + 1 < len(chunk) else 0
+                units += (i + 1) * H * (pairs(b) - below)
+            else:
+                units += H * pairs(b)
         su.append(units)
         p = {"n_seq": len(chunk), "H": H, "seq_units": su, "num_units": units, "causal": causal,
              "window_left": -1, "seq_nq": [lengths[b][0] for b in chunk],
-             "seq_nk": [lengths[b][1] for b in chunk]}
+             "seq_nk": [lengths[b][1] for b in chunk], "level_order": level}
         launches.append((p, {s: lengths[b] for s, b in enumerate(chunk)}))
     return launches, order
 
@@ -178,3 +193,22 @@ def test_planted_mistake_in_the_window_start_is_caught():
             check_units(bad, {0: (1000, 1000)})
     finally:
         globals()["decode"] = orig
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_ragged_causal_batches_in_query_pair_order(seed):
+    """Causal ragged batches with N_q = N_k in every sequence: the launch takes the units of all
+    sequences by query pair, highest first -- heaviest first, since a causal pair's key tiles
+    depend on its index only -- and still every (sequence, head, pair) exactly once."""
+    rng = random.Random(300 + seed)
+    n = rng.choice([1, 2, 5, 16, 64, 70])
+    lengths = [(m, m) for m in (rng.randint(1, 2500) for _ in range(n))]
+    H = rng.randint(1, 4)
+    launches, order = varlen_params(lengths, H, True)
+    for p, problems in launches:
+        assert p["level_order"]
+        check_units(p, problems)
+        qps = [decode(u, p)["qp"] for u in range(p["num_units"])]
+        assert all(a >= b for a, b in zip(qps, qps[1:])), "units not in non-increasing pair order"
+        weights = [decode(u, p)["nkv1"] for u in range(p["num_units"])]
+        assert all(a >= b for a, b in zip(weights, weights[1:])), "units not heaviest first"
