@@ -258,6 +258,22 @@ __device__ __forceinline__ float row_max(const float (&s)[kBlockN]) {
     return sm100::max3(sm100::max3(m[0], m[1], m[2]), sm100::max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
+// Keeps the scores of keys lo <= c < lim of a row's tile and sets the others to -inf: per
+// 32-key chunk a word with the chunk's visible keys as set bits, then one bit test and one
+// select per key rather than two compares and a select (with one bound, the plain compare
+// is cheaper).
+__device__ __forceinline__ void mask_keys(float (&s)[kBlockN], int lo, int lim) {
+#pragma unroll
+    for (int k = 0; k < kBlockN / 32; ++k) {
+        const int a = min(max(lo - 32 * k, 0), 32), b = min(max(lim - 32 * k, 0), 32);
+        const uint32_t below_b = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+        const uint32_t below_a = a >= 32 ? 0xffffffffu : ((1u << a) - 1u);
+        const uint32_t keep = below_b & ~below_a;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) s[32 * k + c] = ((keep >> c) & 1u) ? s[32 * k + c] : -INFINITY;
+    }
+}
+
 // 2^x for two lanes on the FMA and integer pipes instead of the MUFU unit.
 // Range reduction in the style of Cody and Waite: n = floor(x) by a
 // round-toward-minus-infinity add of 1.5 * 2^23 (n then sits in the low
@@ -868,9 +884,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (fast) {
                     if (need_mask || need_win) {
                         const int lim = CAUSAL ? min(U.Nk - kv0, row + U.off - kv0 + 1) : (U.Nk - kv0);
-                        const int lo = win ? row + U.off - p.window_left - kv0 : 0;
+                        if (win) {
+                            mask_keys(s, row + U.off - p.window_left - kv0, lim);
+                        } else {
 #pragma unroll
-                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim && c >= lo) ? s[c] : -INFINITY;
+                            for (int c = 0; c < kBlockN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+                        }
                     }
                     m_tile = row_max(s) * scale_log2;
                 } else {
@@ -938,8 +957,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (need_mask || need_win) {
                         const int lim = CAUSAL ? min(U.Nk - kv0, row + U.off - kv0 + 1) : (U.Nk - kv0);
+                        if (win) {
+                            mask_keys(s, lo, lim);
+                        } else {
 #pragma unroll
-                        for (int c = 0; c < kBlockN; ++c) s[c] = (c < lim && c >= lo) ? s[c] : -INFINITY;
+                            for (int c = 0; c < kBlockN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+                        }
                     }
                     m_tile = row_max(s) * kLog2e;
                 }

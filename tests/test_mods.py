@@ -94,6 +94,8 @@ WINDOW_CASES = [  # N, Nk, d, causal, window: ranges that skip many key tiles, r
     (700, 2900, 128, True, 257),
     (900, 900, 32, False, 300),       # without causal masking: keys from i - w to the end
     (333, 1400, 64, False, 1),
+    (700, 2900, 64, True, 129),       # the second query tile of most units starts a key tile later
+    (1300, 1300, 32, True, 511),
 ]
 
 
