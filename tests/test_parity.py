@@ -213,6 +213,25 @@ def test_several_waves_of_units(B):
     _full_check(w)
 
 
+@pytest.mark.parametrize("d,dtype,causal", [(64, "fp16", True), (64, "bf16", False), (128, "bf16", True)])
+def test_more_than_32_units_per_cta(d, dtype, causal):
+    """5120 single-pair units on 148 SMs: every CTA runs 34-35 units, every per-unit counter of
+    the barrier protocol wraps its parity many times.  Units are heads here (one 256-row pair
+    per head), and the CTAs' 33rd and later units are heads 4736 and up: those are compared in
+    full, with a sample of the others."""
+    w = Workload("units", B=128, H=40, N=256, d=d, dtype=dtype, causal=causal, seed=60 + d)
+    inp = make_inputs(w)
+    o, lse = _run(inp, w)
+    BH = w.B * w.H
+    rng = np.random.default_rng(7)
+    sel = sorted(set(range(4736, BH)) | set(int(x) for x in rng.integers(0, 4736, size=64)))
+    flat = lambda t: t.reshape(BH, *t.shape[2:])
+    q, k, v = (flat(inp[n])[sel].unsqueeze(0) for n in "qkv")
+    o_ref, l_ref = sdpa_forward(q, k, v, causal=causal, scale=w.scale)
+    assert_close_to_oracle(flat(o.cpu())[sel].unsqueeze(0), flat(lse.cpu())[sel].unsqueeze(0), o_ref, l_ref,
+                           w.torch_dtype, f"units d={d}")
+
+
 RECT = [  # (N query rows, Nk key rows, causal, d, dtype, bias, gate)
     (128, 1024, True, 64, "fp16", False, False),      # prefill chunk against a KV cache
     (1, 777, True, 128, "bf16", False, False),        # decode step
