@@ -199,8 +199,9 @@ def cpu_reference(w, steps: int, warmup: int, rows_per_step: int = 1024):
     return flops / secs / 1e12, sample, cores, 1e3 * secs / max(steps, 1)
 
 
-def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
-    """The same metric through the host-buffer entry point (fwd -> attn_fwd_host): every
+def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops, slopes=None):
+    """The same metric through the host-buffer entry point (fwd -> attn_fwd_host, or
+    attn_fwd_host_ex with the workload's score modifications; ALiBi slopes stay on the device): every
     step copies the step's inputs from pinned host memory to the device, runs the kernel,
     and copies O and lse back to pinned host memory.  Steps alternate between two streams
     with their own staging and host output buffers, so one step's copies run under the
@@ -217,7 +218,8 @@ def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
     def e2e_step(i):
         s = i % 2
         fwd(host["q"], host["k"], host["v"], bias=host["bias"], gate=host["gate"], causal=w.causal, scale=w.scale,
-            out=outs[s][0], lse=outs[s][1], staging=stagings[s], stream=streams[s], sync=False)
+            out=outs[s][0], lse=outs[s][1], staging=stagings[s], stream=streams[s], sync=False,
+            softcap=w.softcap, alibi_slopes=slopes, window_left=w.window_left)
 
     steps = max(4, min(args.steps, 20))
     for i in range(2):
@@ -237,7 +239,12 @@ def run_e2e(args, w, inp_cpu, out, lse, stream, world, flops):
     ms = dist_max(e0.elapsed_time(e1) / steps, world)
     return {"value": whole_job_tflops(world, flops, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
-            "api": "fwd() -> attn_fwd_host (C ABI, pinned host buffers), 2 streams"}
+            "api": "fwd() -> attn_fwd_host%s (C ABI, pinned host buffers), 2 streams" % ("_ex" if has_mods(w) else "")}
+
+
+def has_mods(w) -> bool:
+    """Whether the workload carries score modifications (ALiBi, softcap, left window)."""
+    return w.softcap > 0 or bool(w.alibi) or w.window_left >= 0
 
 
 def launch_percentiles(ms):
@@ -523,14 +530,14 @@ def main():
     lib = load_library()
     views = [nat.make_view(t) for t in (inp["q"], inp["k"], inp["v"], inp["bias"], inp["gate"], out)]
     refs = [None if x is None else ctypes.byref(x) for x in views]
-    has_mods = w.softcap > 0 or w.alibi or w.window_left >= 0
+    mods_on = has_mods(w)
     mods = nat.AttnMods(None if slopes is None else slopes.data_ptr(), float(w.softcap), int(w.window_left))
     args_c = (refs[0], refs[1], refs[2], refs[3], refs[4], int(w.causal), float(w.scale))
     tail_c = (refs[5], lse.data_ptr(), stream.cuda_stream)
     status = []
 
     def step():
-        if has_mods:
+        if mods_on:
             r = lib.attn_fwd_ex(*args_c, ctypes.byref(mods), *tail_c)
         else:
             r = lib.attn_fwd(*args_c, *tail_c)
@@ -574,9 +581,7 @@ def main():
     value = whole_job_tflops(world, flops, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs in, host outputs back, every step
-    # (the host-buffer entry point takes no score modifications: no end-to-end leg for such workloads)
-    has_mods = w.softcap > 0 or w.alibi or w.window_left >= 0
-    e2e = None if (args.no_e2e or has_mods) else run_e2e(args, w, inp_cpu, out, lse, stream, world, flops)
+    e2e = None if args.no_e2e else run_e2e(args, w, inp_cpu, out, lse, stream, world, flops, slopes)
 
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops"]            # burst figure: the kernel is timed alone; fp16 dense rate = bf16's

@@ -24,7 +24,7 @@ DEBUG_LIB_PATH = os.path.join(_PKG, "libattn_debug.so")
 ATTN_F16, ATTN_BF16, ATTN_F32, ATTN_E4M3 = 0, 1, 2, 3
 
 # every function include/attn.h declares
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_fwd_fp8", "attn_bwd", "attn_bwd_ex", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_varlen", "attn_fwd_host", "attn_fwd_host_ex", "attn_fwd_fp8", "attn_bwd", "attn_bwd_ex", "attn_status_string", "attn_last_device_status", "attn_set_wait_limit",
             "attn_debug_inject_stall", "attn_debug_exp2", "attn_build_flags", "attn_version")
 
 
@@ -70,6 +70,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.attn_fwd_host.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, P, ctypes.c_void_p,
                                       P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_host.restype = ctypes.c_int
+        lib.attn_fwd_host_ex.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_float, ctypes.POINTER(AttnMods), P,
+                                         ctypes.c_void_p, P, P, P, P, P, P, ctypes.c_void_p, ctypes.c_void_p]
+        lib.attn_fwd_host_ex.restype = ctypes.c_int
         lib.attn_fwd_fp8.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int,
                                      ctypes.c_float, P, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_fwd_fp8.restype = ctypes.c_int
@@ -291,23 +294,32 @@ class Staging:
 
 
 def attn_fwd_host_raw(q, k, v, bias, gate, causal: bool, scale: float, out, lse, staging: Staging,
-                      stream: int) -> int:
-    """Direct call of attn_fwd_host: host tensors in and out, device staging from ``staging``."""
+                      stream: int, softcap: float = 0.0, alibi_slopes: Optional[torch.Tensor] = None,
+                      window_left: int = -1) -> int:
+    """Direct call of attn_fwd_host (attn_fwd_host_ex with score modifications): host tensors in
+    and out, device staging from ``staging``; ``alibi_slopes`` is a CUDA tensor."""
     lib = load_library()
     hq, hk, hv, hb, hg, ho = (make_view(t) for t in (q, k, v, bias, gate, out))
     dq, dk, dv, db, dg, do = (make_view(t) for t in (staging.q, staging.k, staging.v, staging.bias, staging.gate,
                                                     staging.out))
-    return lib.attn_fwd_host(_ref(hq), _ref(hk), _ref(hv), _ref(hb), _ref(hg), int(bool(causal)), float(scale),
-                             _ref(ho), None if lse is None else lse.data_ptr(),
-                             _ref(dq), _ref(dk), _ref(dv), _ref(db), _ref(dg), _ref(do),
-                             None if lse is None else staging.lse.data_ptr(), stream)
+    lse_h = None if lse is None else lse.data_ptr()
+    lse_d = None if lse is None else staging.lse.data_ptr()
+    if not softcap and alibi_slopes is None and window_left < 0:
+        return lib.attn_fwd_host(_ref(hq), _ref(hk), _ref(hv), _ref(hb), _ref(hg), int(bool(causal)), float(scale),
+                                 _ref(ho), lse_h, _ref(dq), _ref(dk), _ref(dv), _ref(db), _ref(dg), _ref(do),
+                                 lse_d, stream)
+    mods = AttnMods(None if alibi_slopes is None else alibi_slopes.data_ptr(), float(softcap), int(window_left))
+    return lib.attn_fwd_host_ex(_ref(hq), _ref(hk), _ref(hv), _ref(hb), _ref(hg), int(bool(causal)), float(scale),
+                                ctypes.byref(mods), _ref(ho), lse_h, _ref(dq), _ref(dk), _ref(dv), _ref(db),
+                                _ref(dg), _ref(do), lse_d, stream)
 
 
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[torch.Tensor] = None,
         gate: Optional[torch.Tensor] = None, causal: bool = False, scale: Optional[float] = None,
         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
         device: Optional[torch.device] = None, staging: Optional[Staging] = None,
-        stream: Optional[torch.cuda.Stream] = None, sync: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+        stream: Optional[torch.cuda.Stream] = None, sync: bool = True, softcap: float = 0.0,
+        alibi_slopes: Optional[torch.Tensor] = None, window_left: int = -1) -> Tuple[torch.Tensor, torch.Tensor]:
     """The end-to-end call: host tensors in, host tensors out (through attn_fwd_host).
 
     The inputs should be pinned (``tensor.pin_memory()``) for asynchronous
@@ -316,11 +328,13 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[torch.
     Everything is enqueued on ``stream`` (default: the current stream); with
     ``sync`` the call waits for it, else the results are valid once the stream
     has reached the call.  Device tensors are accepted too; then nothing is
-    staged and the device results are returned.
+    staged and the device results are returned.  Score modifications as in attn_fwd
+    (``alibi_slopes`` on the device).
     """
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     if q.is_cuda:
-        return attn_fwd(q, k, v, bias, gate, causal, scale, out, lse, stream)
+        return attn_fwd(q, k, v, bias, gate, causal, scale, out, lse, stream, softcap=softcap,
+                        alibi_slopes=alibi_slopes, window_left=window_left)
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
     if staging is None:
@@ -330,7 +344,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: Optional[torch.
     if lse is None:
         lse = torch.empty(q.shape[:-1], dtype=torch.float32, pin_memory=True)
     st = stream or torch.cuda.current_stream(dev)
-    _check(attn_fwd_host_raw(q, k, v, bias, gate, causal, scale, out, lse, staging, st.cuda_stream))
+    _check(attn_fwd_host_raw(q, k, v, bias, gate, causal, scale, out, lse, staging, st.cuda_stream, softcap,
+                             alibi_slopes, window_left))
     if sync:
         st.synchronize()
     return out, lse

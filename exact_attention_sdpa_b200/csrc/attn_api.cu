@@ -488,6 +488,16 @@ bool same_layout(const attn_tensor_t* a, const attn_tensor_t* b) {
     return true;
 }
 
+// The checks of attn_fwd_ex's score modifications (nullable: none).
+attn_status_t check_mods(const attn_mods_t* mods, const attn_tensor_t* bias, const attn_tensor_t* gate) {
+    if (mods == nullptr) return ATTN_OK;
+    if (!std::isfinite(mods->softcap) || mods->softcap < 0.f) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mods->alibi_slopes) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    const bool on = mods->alibi_slopes != nullptr || mods->softcap > 0.f || mods->window_left >= 0;
+    if (on && (bias != nullptr || gate != nullptr)) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
 // attn_fwd_ex with an optional lse layout (defined below the C entry points)
 attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
                        const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
@@ -521,12 +531,8 @@ attn_status_t fwd_impl(const attn_tensor_t* q, const attn_tensor_t* k, const att
     bool empty = false;
     const attn_status_t st = validate_fwd(q, k, v, bias, gate, scale, out, lse, &empty);
     if (st != ATTN_OK) return st;
-    if (mods != nullptr) {
-        if (!std::isfinite(mods->softcap) || mods->softcap < 0.f) return ATTN_ERR_INVALID_ARG;
-        if ((reinterpret_cast<uintptr_t>(mods->alibi_slopes) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
-        const bool on = mods->alibi_slopes != nullptr || mods->softcap > 0.f || mods->window_left >= 0;
-        if (on && (bias != nullptr || gate != nullptr)) return ATTN_ERR_UNSUPPORTED;
-    }
+    const attn_status_t ms = check_mods(mods, bias, gate);
+    if (ms != ATTN_OK) return ms;
     if (empty) return ATTN_OK;
     const int64_t B = q->shape[0], H = q->shape[1], N = q->shape[2], Nk = k->shape[2], d = q->shape[3];
 
@@ -658,10 +664,22 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
                             const attn_tensor_t* q_dev, const attn_tensor_t* k_dev, const attn_tensor_t* v_dev,
                             const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
                             attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream) {
+    return attn_fwd_host_ex(q, k, v, bias, gate, causal, scale, nullptr, out, lse, q_dev, k_dev, v_dev, bias_dev,
+                            gate_dev, out_dev, lse_dev, stream);
+}
+
+attn_status_t attn_fwd_host_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                               const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                               const attn_mods_t* mods, attn_tensor_t* out, float* lse,
+                               const attn_tensor_t* q_dev, const attn_tensor_t* k_dev, const attn_tensor_t* v_dev,
+                               const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
+                               attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream) {
     // every check before the first copy is enqueued
     if (q_dev == nullptr || k_dev == nullptr || v_dev == nullptr || out_dev == nullptr) return ATTN_ERR_INVALID_ARG;
     bool empty = false;
     attn_status_t st = validate_fwd(q_dev, k_dev, v_dev, bias_dev, gate_dev, scale, out_dev, lse_dev, &empty);
+    if (st != ATTN_OK) return st;
+    st = check_mods(mods, bias_dev, gate_dev);
     if (st != ATTN_OK) return st;
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
     if (!same_layout(q, q_dev) || !same_layout(k, k_dev) || !same_layout(v, v_dev) || !same_layout(out, out_dev) ||
@@ -681,7 +699,7 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
                             cudaMemcpyHostToDevice, stream) != cudaSuccess)
             return ATTN_ERR_CUDA;
     }
-    st = attn_fwd(q_dev, k_dev, v_dev, bias_dev, gate_dev, causal, scale, out_dev, lse_dev, stream);
+    st = fwd_impl(q_dev, k_dev, v_dev, bias_dev, gate_dev, causal, scale, mods, out_dev, lse_dev, nullptr, stream);
     if (st != ATTN_OK) return st;
     // device -> host: O, then lse
     if (cudaMemcpyAsync(out->data, out_dev->data, static_cast<size_t>(span_bytes(out)), cudaMemcpyDeviceToHost,

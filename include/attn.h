@@ -111,7 +111,8 @@ attn_status_t attn_fwd(const attn_tensor_t* q, const attn_tensor_t* k, const att
  *   window_left   >= 0: keys j < i + (Nk - N) - window_left are masked (a left
  *                 sliding window; with causal masking a band of window_left + 1
  *                 keys); negative turns it off
- * Key tiles left of every row's window are still visited (masked, not skipped).
+ * With a window, the key tiles wholly left of the window of a 256-row unit's
+ * first row are skipped; the tiles the window's edge cuts are masked.
  */
 typedef struct {
     const float* alibi_slopes;
@@ -194,6 +195,21 @@ attn_status_t attn_fwd_host(const attn_tensor_t* q, const attn_tensor_t* k, cons
                             const attn_tensor_t* q_dev, const attn_tensor_t* k_dev, const attn_tensor_t* v_dev,
                             const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
                             attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream);
+
+/*
+ * attn_fwd_host_ex -- attn_fwd_host with score modifications (`mods` nullable:
+ * none), applied as attn_fwd_ex applies them.  mods->alibi_slopes, when given,
+ * points to DEVICE memory (H fp32), like the staging buffers; it is read by the
+ * kernel, not copied.  The checks of attn_fwd_ex's mods run with the others,
+ * before any copy is enqueued.  attn_fwd_host(...) is attn_fwd_host_ex with
+ * mods = NULL.
+ */
+attn_status_t attn_fwd_host_ex(const attn_tensor_t* q, const attn_tensor_t* k, const attn_tensor_t* v,
+                               const attn_tensor_t* bias, const attn_tensor_t* gate, int causal, float scale,
+                               const attn_mods_t* mods, attn_tensor_t* out, float* lse,
+                               const attn_tensor_t* q_dev, const attn_tensor_t* k_dev, const attn_tensor_t* v_dev,
+                               const attn_tensor_t* bias_dev, const attn_tensor_t* gate_dev,
+                               attn_tensor_t* out_dev, float* lse_dev, cudaStream_t stream);
 
 /*
  * attn_bwd -- gradients of attn_fwd (without bias or gate) for an upstream dO:

@@ -236,6 +236,27 @@ def test_host_entry_applies_device_checks_and_null_rules(lib):
     assert r == nat.ATTN_ERR_INVALID_ARG
 
 
+def test_host_entry_checks_score_modifications_before_any_copy(lib):
+    q, k, v, o = _qkv()
+    st = _FakeStaging(*_qkv()[:3])
+    assert nat.attn_fwd_host_raw(q, k, v, None, None, True, 0.125, o, None, st, 0,
+                                 softcap=-1.0) == nat.ATTN_ERR_INVALID_ARG
+    assert nat.attn_fwd_host_raw(q, k, v, None, None, True, 0.125, o, None, st, 0,
+                                 softcap=float("nan")) == nat.ATTN_ERR_INVALID_ARG
+    bias = torch.zeros(2, 64, 64, dtype=torch.float16)
+    st_b = _FakeStaging(*_qkv()[:3], bias=torch.zeros(2, 64, 64, dtype=torch.float16))
+    assert nat.attn_fwd_host_raw(q, k, v, bias, None, True, 0.125, o, None, st_b, 0,
+                                 window_left=10) == nat.ATTN_ERR_UNSUPPORTED
+    # a misaligned slopes pointer (never dereferenced: rejected first)
+    slopes = torch.zeros(4, dtype=torch.float32)
+    views = [nat.make_view(t) for t in (q, k, v, o, st.q, st.k, st.v, st.out)]
+    refs = [ctypes.byref(x) for x in views]
+    mods = nat.AttnMods(slopes.data_ptr() + 2, 0.0, -1)
+    r = lib.attn_fwd_host_ex(refs[0], refs[1], refs[2], None, None, 1, 0.125, ctypes.byref(mods), refs[3], None,
+                             refs[4], refs[5], refs[6], None, None, refs[7], None, None)
+    assert r == nat.ATTN_ERR_INVALID_ARG
+
+
 def test_host_entry_empty_problem_is_ok(lib):
     q = torch.zeros(1, 2, 0, 64, dtype=torch.float16)
     st = _FakeStaging(q.clone(), q.clone(), q.clone())

@@ -1,5 +1,5 @@
-"""The end-to-end entry point with host buffers (attn_fwd_host, reached through
-fwd()): host inputs are copied to device staging buffers, the same kernel runs,
+"""The end-to-end entry point with host buffers (attn_fwd_host, and attn_fwd_host_ex with
+score modifications, reached through fwd()): host inputs are copied to device staging buffers, the same kernel runs,
 O and lse come back to host memory.  Results must equal the device-path call bit
 for bit and the oracle within tolerance; two streams with their own staging
 buffers may run calls concurrently."""
@@ -34,6 +34,28 @@ def test_host_path_matches_device_path_and_oracle(name):
     o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], bias=inp["bias"], gate=inp["gate"],
                                 causal=w.causal, scale=w.scale)
     assert_close_to_oracle(o_h, l_h, o_ref, l_ref, w.torch_dtype, name + "-host")
+
+
+@pytest.mark.parametrize("softcap,alibi,window", [(30.0, True, -1), (0.0, False, 300), (2.0, False, 129)])
+def test_host_path_with_score_modifications(softcap, alibi, window):
+    """attn_fwd_host_ex: the same kernel as attn_fwd_ex on the staged inputs (ALiBi slopes on
+    the device), so the host results equal the device path's bit for bit, and the oracle's."""
+    w = Workload("hm", B=2, H=4, N=700, d=64, dtype="bf16", causal=True, seed=55)
+    inp = make_inputs(w)
+    h = _pinned(inp)
+    dev = torch.device("cuda")
+    slopes = torch.tensor([2.0 ** (-8.0 * (i + 1) / w.H) for i in range(w.H)], dtype=torch.float32) if alibi else None
+    sd = None if slopes is None else slopes.to(dev)
+    kw = dict(causal=True, scale=w.scale, softcap=softcap, alibi_slopes=sd, window_left=window)
+    o_h, l_h = fwd(h["q"], h["k"], h["v"], **kw)
+    assert not o_h.is_cuda
+    o_d, l_d = attn_fwd(inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev), **kw)
+    torch.cuda.synchronize()
+    assert last_device_status() == 0
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
+    o_ref, l_ref = sdpa_forward(inp["q"], inp["k"], inp["v"], causal=True, scale=w.scale, softcap=softcap,
+                                alibi_slopes=slopes, window_left=window)
+    assert_close_to_oracle(o_h, l_h, o_ref, l_ref, w.torch_dtype, "host path with modifications")
 
 
 def test_two_streams_pipeline():
